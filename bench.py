@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Throughput of the MoE boundary step: router gate + RMSNorm/NVFP4 + post-expert combine.
+
+Workload (one step, per GPU): T=8192 tokens, H=8192, E=256 experts, top-8,
+router logits FP32 N(0, 2), 5% of tokens masked, 1% of expert slots invalid,
+expert outputs [T*8, H] BF16 -- synthetic, seeded, resident in HBM.  The
+three calls go through the library's C ABI on one stream.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  `value` is tokens/s over all ranks (weak
+scaling: every rank runs its own batch of 8192 tokens).  The per-step inputs
+(1.2 GB) are larger than the 126 MB L2, so no flush runs between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "prefill"
+METRIC = "tokens/s of route+norm-quant+combine at 8192 tok, H=8192; HBM GB/s vs 8 TB/s"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def bytes_per_token(H, E, k):
+    """Algorithmic bytes per token, counted once (reads + writes)."""
+    route = 4 * E + 1 + 8 * k                       # logits, mask, ids + weights
+    norm_quant = 2 * H + H // 2 + H // 16           # x, packed codes, scales
+    combine = 2 * k * H + 8 * k + 2 * H             # k expert rows, idx + weights, out
+    return route, norm_quant, combine
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_step(case_host, tokens):
+    """The oracle on a sample of the workload's tokens (all three stages)."""
+    import oracle
+    c = case_host
+    ids, w = oracle.route(c["logits"][tokens], c["bias"], c["mask"][tokens], c["k"])
+    oracle.norm_quant(c["x"][tokens], len(tokens), c["H"], 1, c["norm_w"], c["gc"], c["eps"],
+                      c["gs"])
+    idx = c["row_idx"][tokens]
+    valid = (idx >= 0) & (idx < c["R"])
+    rows = np.unique(idx[valid])
+    remap = np.full(idx.shape, -1, np.int32)
+    remap[valid] = np.searchsorted(rows, idx[valid]).astype(np.int32)
+    sub = c["expert_rows"](rows)
+    oracle.combine(sub, sub.shape[0], remap, w, c["post_w"], c["post_gc"], c["eps"])
+
+
+def host_sample(case, n_tokens, seed=0):
+    """Copy to the host what the oracle needs for a sample of tokens."""
+    from expert_combine_b200 import synth
+    rng = np.random.default_rng(seed)
+    tokens = np.sort(rng.choice(case.T, size=n_tokens, replace=False))
+    tk = torch.as_tensor(tokens, device=case.logits.device)
+    idx = synth.host(case.row_idx)
+    sel_rows = idx[tokens]
+    need = np.unique(sel_rows[(sel_rows >= 0) & (sel_rows < case.R)])
+    rows_host = synth.host(case.expert_out.index_select(
+        0, torch.as_tensor(need, device=case.logits.device, dtype=torch.int64)))
+    logits = np.full((case.T, case.E), np.nan, np.float32)
+    logits[tokens] = synth.host(case.logits.index_select(0, tk))
+    x = np.zeros((case.T, case.H), np.uint16)
+    x[tokens] = synth.host(case.x_logical().index_select(0, tk))
+
+    def expert_rows(rows):
+        pos = np.searchsorted(need, rows)
+        return rows_host[pos]
+
+    return tokens, dict(logits=logits, bias=synth.host(case.bias), mask=synth.host(case.mask),
+                        k=case.k, x=x, H=case.H, norm_w=synth.host(case.norm_w), gc=case.gc,
+                        eps=case.eps, gs=float(synth.host(case.gs)[0]), row_idx=idx, R=case.R,
+                        expert_rows=expert_rows, post_w=synth.host(case.post_w),
+                        post_gc=case.post_gc)
+
+
+def time_oracle(case_host, tokens, budget_s=15.0):
+    import oracle
+    cores = oracle.get_threads()
+    t0 = time.perf_counter()
+    oracle_step(case_host, tokens)
+    one = time.perf_counter() - t0
+    reps = max(1, min(20, int(budget_s / max(one, 1e-3))))
+    times = [one]
+    for _ in range(reps - 1):
+        t0 = time.perf_counter()
+        oracle_step(case_host, tokens)
+        times.append(time.perf_counter() - t0)
+    med = statistics.median(times)
+    return len(tokens) / med, cores, reps, med
+
+
+# ---------------------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from expert_combine_b200 import synth
+    case = synth.make_case(WORKLOAD, device="cuda" if torch.cuda.is_available() else "cpu")
+    n_sample = 256
+    tokens, ch = host_sample(case, n_sample, seed=1)
+    import oracle
+    cores = oracle.get_threads()
+    for _ in range(args.warmup):
+        oracle_step(ch, tokens)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(ch, tokens)
+        times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = len(tokens) / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "prefill T=8192 H=8192 E=256 k=8 (oracle on a token sample)",
+                   "sample_tokens": n_sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_sample} of 8192 tokens per step, all three stages"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import expert_combine_b200 as eb
+    from expert_combine_b200 import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    eb.load()
+    case = synth.make_case(WORKLOAD, device=dev, seed=synth.SEEDS[WORKLOAD] + rank)
+    T, H, E, k = case.T, case.H, case.E, case.k
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    packed = torch.empty(T, H // 2, dtype=torch.uint8, device=dev)
+    sf = torch.empty(T, H // 16, dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = {}
+
+    def step(timed_combine=None):
+        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
+                            sf=sf)
+        if timed_combine is not None:
+            timed_combine[0].record(stream)
+        eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
+                          case.eps, out=out)
+        if timed_combine is not None:
+            timed_combine[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if eb.device_status() != 0:
+        raise RuntimeError("a kernel reported a wait timeout during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    cmb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        # keep the timed region long enough for the clock sampler to see it
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step(cmb[i])
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    combine_ms = sum(a.elapsed_time(b) for a, b in cmb) / args.steps
+    step_ms_max = max_over_ranks(step_ms, world)
+    ms_per_step = step_ms_max / args.steps
+
+    # algorithmic bytes
+    b_route, b_nq, b_cmb = bytes_per_token(H, E, k)
+    idx_h = synth.host(case.row_idx)
+    valid_slots = int(((idx_h >= 0) & (idx_h < case.R)).sum())
+    valid_tokens = int(synth.host(case.mask).sum())
+    cmb_bytes_nominal = T * b_cmb
+    cmb_bytes_net = valid_slots * 2 * H + T * (8 * k + 2 * H)
+    step_bytes_nominal = T * (b_route + b_nq + b_cmb)
+    peak, peak_kind = measured_peaks()
+    achieved_cmb = cmb_bytes_net / (combine_ms * 1e-3) / 1e9
+
+    # end to end through the same calls with host buffers (pinned), copies inside
+    e2e = run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps=max(2, min(args.steps, 5)))
+
+    tokens_per_s = T * world / (ms_per_step * 1e-3)
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            n_sample = 512
+            tokens, ch = host_sample(case, n_sample, seed=2)
+            v, cores, reps, med = time_oracle(ch, tokens)
+            cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": f"{n_sample} of 8192 tokens (all three stages), median of {reps} "
+                             f"runs of {med:.2f} s"}
+        clk = clocks.summary()
+        result = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "prefill T=8192 H=8192 E=256 k=8 (route+norm-quant+combine)",
+                       "tokens_per_rank": T, "hidden": H, "experts": E, "top_k": k,
+                       "expert_rows": case.R, "valid_tokens": valid_tokens,
+                       "valid_slots": valid_slots, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (1.2 GB per step), no flush"},
+            "hbm": {"step_bytes_nominal": step_bytes_nominal,
+                    "step_gbs": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9,
+                    "frac_of_8tbs": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+                    "frac_of_measured": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9 / peak},
+            "roofline": {"kernel": "combine", "bound": "hbm", "achieved": achieved_cmb,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved_cmb / peak, "traffic": None,
+                         "bytes_per_launch": cmb_bytes_net,
+                         "bytes_per_launch_nominal": cmb_bytes_nominal,
+                         "avg_launch_ms": combine_ms},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                       "reasons": clk["reasons"], "samples": clk["samples"],
+                       "timed_wall_s": t_wall},
+        }
+        print(json.dumps(result), flush=True)
+    if eb.device_status() != 0:
+        raise RuntimeError("a kernel reported a wait timeout")
+    return result
+
+
+def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps):
+    """Host inputs (pinned) -> device -> the three calls -> host outputs, per step."""
+    T, H, k = case.T, case.H, case.k
+    h_in = {name: t.detach().cpu().pin_memory() for name, t in
+            (("logits", case.logits), ("mask", case.mask), ("x", case.x),
+             ("expert", case.expert_out), ("idx", case.row_idx))}
+    h_out = {name: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for name, t in
+             (("ids", ids), ("w", w), ("packed", packed), ("sf", sf), ("out", out))}
+    d_in = {"logits": case.logits, "mask": case.mask, "x": case.x,
+            "expert": case.expert_out, "idx": case.row_idx}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def one():
+        for name, h in h_in.items():
+            d_in[name].copy_(h, non_blocking=True)
+        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
+                            sf=sf)
+        eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
+                          case.eps, out=out)
+        for name, d in (("ids", ids), ("w", w), ("packed", packed), ("sf", sf), ("out", out)):
+            h_out[name].copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return {"value": T / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = init_dist() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        run_ours(args, world, rank, local)
+        return 0
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

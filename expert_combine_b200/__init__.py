@@ -1,1 +1,29 @@
+"""B200-native per-token MoE boundary: router gate, RMSNorm + NVFP4, expert combine, residual join.
 
+Thin Python binding over the C ABI of ``libmoe_boundary.so`` (declared in
+``include/moe_boundary.h``).  This package only marshals arguments: it checks
+dtypes/devices, allocates outputs with torch when the caller passes none, and
+enqueues the library call on torch's current CUDA stream.  Every step of the
+boundary runs in the library's CUDA kernels; there is no host fallback.  If the
+library cannot be loaded the calls raise.
+"""
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    MoEBoundaryError,
+    STAGE_COMBINE,
+    STAGE_COMBINE_JOIN,
+    STAGE_JOIN,
+    STAGE_NORM_QUANT,
+    STAGE_ROUTE,
+    device_status,
+    expert_combine,
+    expert_combine_join,
+    last_error,
+    lib_path,
+    load,
+    moe_route,
+    norm_quant_nvfp4,
+    residual_join,
+    supported,
+)

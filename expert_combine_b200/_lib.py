@@ -1,0 +1,240 @@
+"""ctypes binding of libmoe_boundary.so (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+STAGE_ROUTE = 0
+STAGE_NORM_QUANT = 1
+STAGE_COMBINE = 2
+STAGE_JOIN = 3
+STAGE_COMBINE_JOIN = 4
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MoEBoundaryError(RuntimeError):
+    """A library call returned an error status."""
+
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn} failed with status {status}: {message}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load() -> ctypes.CDLL:
+    """Load the library, building it first when it is missing or stale.
+
+    Raises when it can be neither found nor built: there is no fallback path.
+    """
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if _build.is_stale():
+                try:
+                    _build.build()
+                except Exception as exc:   # no nvcc, compile error, ...
+                    if not os.path.exists(path):
+                        raise RuntimeError(
+                            f"libmoe_boundary.so is missing and could not be built: {exc}") from exc
+            lib = ctypes.CDLL(path)
+            P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+            sigs = {
+                "moe_route": [P, P, P, i32, i32, i32, P, P, P],
+                "norm_quant_nvfp4": [P, i32, i32, i32, P, f32, f32, P, P, P, P],
+                "expert_combine": [P, i64, i32, P, P, i32, i32, P, f32, f32, P, P],
+                "residual_join": [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32, P],
+                "expert_combine_join": [P, i64, i32, P, P, i32, i32, P, f32, f32, P, P, P, f32, f32,
+                                        f32, P, f32, f32, P, P],
+                "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
+                "mb_last_error": [],
+                "mb_device_status": [],
+            }
+            for name, args in sigs.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = ctypes.c_char_p if name == "mb_last_error" else ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def last_error() -> str:
+    return load().mb_last_error().decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MoEBoundaryError(fn, status, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+def supported(stage: int, T: int = 1, H: int = 16, E: int = 1, k: int = 1, tp: int = 1) -> bool:
+    return bool(load().moe_boundary_supported(stage, T, H, E, k, tp))
+
+
+def device_status() -> int:
+    """Read and clear the library's device-side timeout flags (0 = none)."""
+    v = load().mb_device_status()
+    if v < 0:
+        raise MoEBoundaryError("mb_device_status", v, last_error())
+    return v
+
+
+def moe_route(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor, k: int,
+              topk_ids: Optional[torch.Tensor] = None, topk_weights: Optional[torch.Tensor] = None,
+              stream=None):
+    """Sigmoid router gate -> (topk_ids int32 [T, k], topk_weights float32 [T, k])."""
+    _want(logits, torch.float32, "logits")
+    _want(bias, torch.float32, "bias")
+    _want(token_mask, torch.uint8, "token_mask")
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    if topk_weights is None:
+        topk_weights = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    _want(topk_ids, torch.int32, "topk_ids")
+    _want(topk_weights, torch.float32, "topk_weights")
+    if bias.numel() != E or token_mask.numel() != T or topk_ids.shape != (T, k) \
+            or topk_weights.shape != (T, k):
+        raise ValueError("moe_route: shape mismatch")
+    _check("moe_route", load().moe_route(_ptr(logits), _ptr(bias), _ptr(token_mask), T, E, k,
+                                         _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+    return topk_ids, topk_weights
+
+
+def norm_quant_nvfp4(x: torch.Tensor, num_tokens: int, norm_w: torch.Tensor, gain_center: float,
+                     eps: float, global_scale: torch.Tensor, tp: int = 1,
+                     packed: Optional[torch.Tensor] = None, sf: Optional[torch.Tensor] = None,
+                     stream=None):
+    """RMSNorm + NVFP4 -> (packed uint8 [M, H/2], sf uint8 [M, H/16]).
+
+    ``x`` is [M, H] (tp == 1) or the rank-block [tp, M, H/tp] (any shape with
+    M * H elements in that order).
+    """
+    _want(x, torch.bfloat16, "x")
+    _want(norm_w, torch.bfloat16, "norm_w")
+    _want(global_scale, torch.float32, "global_scale")
+    H = norm_w.numel()
+    M = int(num_tokens)
+    if x.numel() != M * H:
+        raise ValueError("norm_quant_nvfp4: x must hold num_tokens * H elements")
+    if packed is None:
+        packed = torch.empty(M, H // 2, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(M, H // 16, dtype=torch.uint8, device=x.device)
+    _want(packed, torch.uint8, "packed")
+    _want(sf, torch.uint8, "sf")
+    if packed.numel() != M * (H // 2) or sf.numel() != M * (H // 16):
+        raise ValueError("norm_quant_nvfp4: output shape mismatch")
+    _check("norm_quant_nvfp4",
+           load().norm_quant_nvfp4(_ptr(x), M, H, tp, _ptr(norm_w), float(gain_center), float(eps),
+                                   _ptr(global_scale), _ptr(packed), _ptr(sf), _stream(stream)))
+    return packed, sf
+
+
+def expert_combine(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
+                   weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
+                   out: Optional[torch.Tensor] = None, stream=None):
+    """Post-expert RMSNorm + weighted top-k combine -> out bf16 [T, H]."""
+    _want(expert_out, torch.bfloat16, "expert_out")
+    _want(row_idx, torch.int32, "row_idx")
+    _want(weights, torch.float32, "weights")
+    _want(norm_w, torch.bfloat16, "norm_w")
+    H = norm_w.numel()
+    T, k = row_idx.shape
+    if weights.shape != (T, k) or expert_out.shape[-1] != H:
+        raise ValueError("expert_combine: shape mismatch")
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=row_idx.device)
+    _want(out, torch.bfloat16, "out")
+    _check("expert_combine",
+           load().expert_combine(_ptr(expert_out), int(num_rows), H, _ptr(row_idx), _ptr(weights),
+                                 T, k, _ptr(norm_w), float(gain_center), float(eps), _ptr(out),
+                                 _stream(stream)))
+    return out
+
+
+def residual_join(residual: torch.Tensor, branch: torch.Tensor, gain: torch.Tensor, alpha: float,
+                  beta: float, eps: float, next_w: Optional[torch.Tensor] = None,
+                  next_gc: float = 1.0, next_eps: float = 1e-6,
+                  next_prenorm: Optional[torch.Tensor] = None, stream=None):
+    """Gated residual join (residual updated in place) -> next_prenorm or None."""
+    _want(residual, torch.float32, "residual")
+    _want(branch, torch.bfloat16, "branch")
+    _want(gain, torch.bfloat16, "gain")
+    T, H = residual.shape
+    if branch.shape != (T, H) or gain.numel() != H:
+        raise ValueError("residual_join: shape mismatch")
+    if next_w is not None:
+        _want(next_w, torch.bfloat16, "next_w")
+        if next_prenorm is None:
+            next_prenorm = torch.empty(T, H, dtype=torch.bfloat16, device=residual.device)
+        _want(next_prenorm, torch.bfloat16, "next_prenorm")
+    _check("residual_join",
+           load().residual_join(_ptr(residual), _ptr(branch), _ptr(gain), float(alpha),
+                                float(beta), float(eps), _ptr(next_w), float(next_gc),
+                                float(next_eps), _ptr(next_prenorm), T, H, _stream(stream)))
+    return next_prenorm
+
+
+def expert_combine_join(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
+                        weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float,
+                        eps: float, residual: torch.Tensor, gain: torch.Tensor, alpha: float,
+                        beta: float, join_eps: float, next_w: Optional[torch.Tensor] = None,
+                        next_gc: float = 1.0, next_eps: float = 1e-6,
+                        out: Optional[torch.Tensor] = None,
+                        next_prenorm: Optional[torch.Tensor] = None, stream=None):
+    """Combine fused with the residual join -> (out or None, next_prenorm or None)."""
+    _want(expert_out, torch.bfloat16, "expert_out")
+    _want(row_idx, torch.int32, "row_idx")
+    _want(weights, torch.float32, "weights")
+    _want(norm_w, torch.bfloat16, "norm_w")
+    _want(residual, torch.float32, "residual")
+    _want(gain, torch.bfloat16, "gain")
+    H = norm_w.numel()
+    T, k = row_idx.shape
+    if weights.shape != (T, k) or residual.shape != (T, H) or gain.numel() != H:
+        raise ValueError("expert_combine_join: shape mismatch")
+    if out is not None:
+        _want(out, torch.bfloat16, "out")
+    if next_w is not None:
+        _want(next_w, torch.bfloat16, "next_w")
+        if next_prenorm is None:
+            next_prenorm = torch.empty(T, H, dtype=torch.bfloat16, device=residual.device)
+    _check("expert_combine_join",
+           load().expert_combine_join(_ptr(expert_out), int(num_rows), H, _ptr(row_idx),
+                                      _ptr(weights), T, k, _ptr(norm_w), float(gain_center),
+                                      float(eps), _ptr(out), _ptr(residual), _ptr(gain),
+                                      float(alpha), float(beta), float(join_eps), _ptr(next_w),
+                                      float(next_gc), float(next_eps), _ptr(next_prenorm),
+                                      _stream(stream)))
+    return out, next_prenorm

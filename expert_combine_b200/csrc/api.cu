@@ -1,0 +1,200 @@
+// api.cu -- the C ABI (include/moe_boundary.h): argument checks, status codes
+// and launches.  No allocation, no synchronisation, no host fallback.
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/moe_boundary.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace mb {
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return MB_OK;
+    return fail(MB_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_once[kMaxDevices];
+
+bool hidden_ok(int H) { return H > 0 && H % 16 == 0 && H <= kMaxHidden; }
+
+}  // namespace
+
+const DeviceInfo& device_info() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) dev = 0;
+    std::call_once(g_once[dev], [dev] {
+        int sms = 148, smem = 227 * 1024;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        g_info[dev].sm_count = sms;
+        g_info[dev].max_smem_optin = smem;
+    });
+    return g_info[dev];
+}
+
+}  // namespace mb
+
+using namespace mb;
+
+extern "C" {
+
+const char* mb_last_error(void) { return t_last_error; }
+
+int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp) {
+    if (T < 0) return 0;
+    switch (stage) {
+        case MB_STAGE_ROUTE:
+            return (k >= 1 && k <= kMaxTopK && E >= k && E <= kMaxExperts) ? 1 : 0;
+        case MB_STAGE_NORM_QUANT:
+            return (hidden_ok(H) && tp >= 1 && H % tp == 0 && (H / tp) % 16 == 0) ? 1 : 0;
+        case MB_STAGE_COMBINE:
+        case MB_STAGE_COMBINE_JOIN:
+            return (hidden_ok(H) && k >= 1 && k <= kMaxTopK) ? 1 : 0;
+        case MB_STAGE_JOIN:
+            return hidden_ok(H) ? 1 : 0;
+        default:
+            return 0;
+    }
+}
+
+int moe_route(const float* logits, const float* bias, const uint8_t* token_mask, int T, int E, int k,
+              int32_t* topk_ids, float* topk_weights, void* stream) {
+    if (T < 0 || E < 0 || k < 0) return fail(MB_ERR_INVALID_ARG, "moe_route: negative size");
+    if (!moe_boundary_supported(MB_STAGE_ROUTE, T, 0, E, k, 1))
+        return fail(MB_ERR_UNSUPPORTED, "moe_route: needs 1 <= k <= %d and k <= E <= %d (k=%d, E=%d)",
+                    kMaxTopK, kMaxExperts, k, E);
+    if (T == 0) return MB_OK;
+    if (!logits || !bias || !token_mask || !topk_ids || !topk_weights)
+        return fail(MB_ERR_INVALID_ARG, "moe_route: null pointer");
+    if (!aligned16(logits) || !aligned16(bias) || !aligned16(token_mask) || !aligned16(topk_ids) ||
+        !aligned16(topk_weights))
+        return fail(MB_ERR_INVALID_ARG, "moe_route: pointers must be 16-byte aligned");
+    return cuda_status(launch_route(logits, bias, token_mask, T, E, k, topk_ids, topk_weights,
+                                    static_cast<cudaStream_t>(stream)),
+                       "moe_route");
+}
+
+int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* norm_w, float gain_center,
+                     float eps, const float* global_scale, uint8_t* packed, uint8_t* sf, void* stream) {
+    if (M < 0 || H < 0 || tp < 0) return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: negative size");
+    if (tp == 0 || H % 16 != 0 || H % tp != 0 || (H / tp) % 16 != 0)
+        return fail(MB_ERR_INVALID_ARG,
+                    "norm_quant_nvfp4: needs H %% 16 == 0, tp >= 1, H %% tp == 0, (H/tp) %% 16 == 0 "
+                    "(H=%d, tp=%d)", H, tp);
+    if (!moe_boundary_supported(MB_STAGE_NORM_QUANT, M, H, 0, 0, tp))
+        return fail(MB_ERR_UNSUPPORTED, "norm_quant_nvfp4: H=%d outside 16..%d", H, kMaxHidden);
+    if (M == 0) return MB_OK;
+    if (!x || !norm_w || !global_scale || !packed || !sf)
+        return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: null pointer");
+    if (!aligned16(x) || !aligned16(norm_w) || !aligned16(packed) || !aligned16(sf) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+        return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: pointers must be 16-byte aligned");
+    return cuda_status(launch_norm_quant(x, M, H, tp, norm_w, gain_center, eps, global_scale, packed, sf,
+                                         static_cast<cudaStream_t>(stream)),
+                       "norm_quant_nvfp4");
+}
+
+static int check_combine(const char* fn, const uint16_t* expert_out, int64_t num_rows, int H,
+                         const int32_t* row_idx, const float* weights, int T, int k,
+                         const uint16_t* norm_w) {
+    if (T < 0 || H < 0 || k < 0 || num_rows < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (H % 16 != 0) return fail(MB_ERR_INVALID_ARG, "%s: H %% 16 != 0 (H=%d)", fn, H);
+    if (!moe_boundary_supported(MB_STAGE_COMBINE, T, H, 0, k, 1))
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs 16 <= H <= %d and 1 <= k <= %d (H=%d, k=%d)", fn,
+                    kMaxHidden, kMaxTopK, H, k);
+    if (T == 0) return MB_OK;
+    if ((num_rows > 0 && !expert_out) || !row_idx || !weights || !norm_w)
+        return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(expert_out) || !aligned16(row_idx) || !aligned16(weights) || !aligned16(norm_w))
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return MB_OK;
+}
+
+static int check_join(const char* fn, float* residual, const uint16_t* gain, const uint16_t* next_w,
+                      uint16_t* next_prenorm) {
+    if (!residual || !gain) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if ((next_w == nullptr) != (next_prenorm == nullptr))
+        return fail(MB_ERR_INVALID_ARG, "%s: next_w and next_prenorm must both be set or both be NULL", fn);
+    if (!aligned16(residual) || !aligned16(gain) || !aligned16(next_w) || !aligned16(next_prenorm))
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return MB_OK;
+}
+
+int expert_combine(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                   const float* weights, int T, int k, const uint16_t* norm_w, float gain_center, float eps,
+                   uint16_t* out, void* stream) {
+    int st = check_combine("expert_combine", expert_out, num_rows, H, row_idx, weights, T, k, norm_w);
+    if (st != MB_OK || T == 0) return st;
+    if (!out) return fail(MB_ERR_INVALID_ARG, "expert_combine: null pointer");
+    if (!aligned16(out)) return fail(MB_ERR_INVALID_ARG, "expert_combine: pointers must be 16-byte aligned");
+    JoinArgs none{};
+    return cuda_status(launch_combine(expert_out, num_rows, H, row_idx, weights, T, k, norm_w, gain_center,
+                                      eps, out, none, static_cast<cudaStream_t>(stream)),
+                       "expert_combine");
+}
+
+int residual_join(float* residual, const uint16_t* branch, const uint16_t* gain, float alpha, float beta,
+                  float eps, const uint16_t* next_w, float next_gc, float next_eps, uint16_t* next_prenorm,
+                  int T, int H, void* stream) {
+    if (T < 0 || H < 0) return fail(MB_ERR_INVALID_ARG, "residual_join: negative size");
+    if (H % 16 != 0) return fail(MB_ERR_INVALID_ARG, "residual_join: H %% 16 != 0 (H=%d)", H);
+    if (!moe_boundary_supported(MB_STAGE_JOIN, T, H, 0, 0, 1))
+        return fail(MB_ERR_UNSUPPORTED, "residual_join: H=%d outside 16..%d", H, kMaxHidden);
+    if (T == 0) return MB_OK;
+    int st = check_join("residual_join", residual, gain, next_w, next_prenorm);
+    if (st != MB_OK) return st;
+    if (!branch) return fail(MB_ERR_INVALID_ARG, "residual_join: null pointer");
+    if (!aligned16(branch)) return fail(MB_ERR_INVALID_ARG, "residual_join: pointers must be 16-byte aligned");
+    JoinArgs j{residual, gain, alpha, beta, eps, next_w, next_gc, next_eps, next_prenorm};
+    return cuda_status(launch_residual_join(branch, T, H, j, static_cast<cudaStream_t>(stream)),
+                       "residual_join");
+}
+
+int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                        const float* weights, int T, int k, const uint16_t* norm_w, float gain_center,
+                        float eps, uint16_t* out, float* residual, const uint16_t* gain, float alpha,
+                        float beta, float join_eps, const uint16_t* next_w, float next_gc, float next_eps,
+                        uint16_t* next_prenorm, void* stream) {
+    int st = check_combine("expert_combine_join", expert_out, num_rows, H, row_idx, weights, T, k, norm_w);
+    if (st != MB_OK || T == 0) return st;
+    st = check_join("expert_combine_join", residual, gain, next_w, next_prenorm);
+    if (st != MB_OK) return st;
+    if (!aligned16(out))
+        return fail(MB_ERR_INVALID_ARG, "expert_combine_join: pointers must be 16-byte aligned");
+    JoinArgs j{residual, gain, alpha, beta, join_eps, next_w, next_gc, next_eps, next_prenorm};
+    return cuda_status(launch_combine(expert_out, num_rows, H, row_idx, weights, T, k, norm_w, gain_center,
+                                      eps, out, j, static_cast<cudaStream_t>(stream)),
+                       "expert_combine_join");
+}
+
+int mb_device_status(void) {
+    unsigned int v = 0u, zero = 0u;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_wait_timeout, sizeof(v));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_wait_timeout, &zero, sizeof(zero));
+    if (e != cudaSuccess) {
+        fail(MB_ERR_CUDA, "mb_device_status: %s", cudaGetErrorString(e));
+        return -1;
+    }
+    return static_cast<int>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,44 @@
+// internal.h -- launchers shared between the kernel files and the C-ABI
+// entry points (host side).  Each returns a cudaError_t from the launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mb {
+
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;
+};
+const DeviceInfo& device_info();   // current device, cached per device
+
+cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
+                         int k, int32_t* ids, float* weights, cudaStream_t s);
+
+cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uint16_t* w, float gc,
+                              float eps, const float* gs, uint8_t* packed, uint8_t* sf,
+                              cudaStream_t s);
+
+struct JoinArgs {
+    float* residual;            // [T, H] FP32 in/out; NULL = no join
+    const uint16_t* gain;       // [H] BF16
+    float alpha, beta, eps;
+    const uint16_t* next_w;     // [H] BF16, NULL = no next prenorm
+    float next_gc, next_eps;
+    uint16_t* next_prenorm;     // [T, H] BF16
+};
+
+cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const int32_t* row_idx,
+                           const float* wt, int T, int k, const uint16_t* w, float gc, float eps,
+                           uint16_t* out, const JoinArgs& join, cudaStream_t s);
+
+cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,
+                                 cudaStream_t s);
+
+// Largest H the row kernels take (16-element blocks, at most 1024 per row).
+constexpr int kMaxHidden = 16384;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 4096;
+
+}  // namespace mb

@@ -1,0 +1,196 @@
+/*
+ * moe_boundary.h -- C ABI of the per-token MoE boundary of a sparse decoder
+ * layer on NVIDIA B200 (sm_100a): router gate, pre-expert RMSNorm fused with
+ * NVFP4 quantisation, post-expert norm + weighted combine, gated residual join.
+ *
+ * Library: libmoe_boundary.so (CUDA runtime only; no PyTorch types).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are DEVICE pointers owned by the caller, row-major and
+ *    contiguous; every base pointer must be 16-byte aligned.  BF16 values are
+ *    passed as uint16_t bit patterns, E4M3 and packed E2M1 as uint8_t.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    only enqueued; nothing is synchronised, allocated or freed.
+ *  - Return value: MB_OK, or an error code.  Arguments are checked before
+ *    anything is enqueued, so on an error nothing runs; mb_last_error()
+ *    returns a message for the calling thread's most recent failure.
+ *  - A call with zero tokens returns MB_OK without launching (the empty-input
+ *    rule of norm_quant_trtllm_nvfp4 on the vLLM API page
+ *    "prepare_trtllm_nvfp4").
+ *  - Floating point: FP32 arithmetic in a fixed order with one IEEE rounding
+ *    per operation; fused multiply-adds only where stated.  Results are
+ *    bitwise reproducible run to run.
+ */
+#ifndef MOE_BOUNDARY_H
+#define MOE_BOUNDARY_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    MB_OK = 0,
+    MB_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer, shape mismatch */
+    MB_ERR_UNSUPPORTED = 2,  /* valid, but outside the sizes the kernels take (see each call)  */
+    MB_ERR_CUDA = 3,         /* the CUDA runtime reported an error while enqueuing             */
+};
+
+/*
+ * moe_route -- sigmoid router gate with selection bias and token mask.
+ *
+ * Source: TensorRT-LLM PR 21356 "Add the Muse Spark Open decoder fast paths",
+ * description, "Routing" (sigmoid, bias, top-k, renormalised weights, picks
+ * sorted with exact ties to the lowest expert id); TensorRT-LLM PR 21042
+ * (router in FP32); lmdeploy PR 4835 "MoE gate v2", commit notes (a required
+ * token mask; invalid tokens produce no routing entries).
+ *
+ * For a valid token t (token_mask[t] != 0):
+ *   s_e = 1 / (1 + exp(-logits[t, e]))          exp: the library's own FP32 exp
+ *   c_e = s_e + bias[e]                          used for selection only
+ *   topk_ids[t, j]     = j-th expert in the order (c descending, id ascending)
+ *   topk_weights[t, j] = s_{id j} / (s_{id 0} + ... + s_{id k-1})
+ * For an invalid token: topk_ids[t, :] = -1, topk_weights[t, :] = 0, and its
+ * logits are not read (they may hold NaN).
+ *
+ *   logits        [T, E] FP32          bias          [E] FP32
+ *   token_mask    [T] uint8 (required) topk_ids      [T, k] int32 (out)
+ *   topk_weights  [T, k] FP32 (out)
+ * Supported: 1 <= k <= 32, k <= E <= 4096.
+ */
+int moe_route(const float* logits, const float* bias, const uint8_t* token_mask, int T, int E,
+              int k, int32_t* topk_ids, float* topk_weights, void* stream);
+
+/*
+ * norm_quant_nvfp4 -- pre-expert RMSNorm fused with NVFP4 quantisation.
+ *
+ * Source: vLLM API page "prepare_trtllm_nvfp4", norm_quant_trtllm_nvfp4 and
+ * _quantize_nvfp4_global_scale; TensorRT-LLM PR 21356, "Numerics" (the gain
+ * centre is added in FP32 and the norm's result is rounded to BF16 once).
+ *
+ * Per token t, over logical x[t, 0..H-1]:
+ *   inv  = 1 / sqrt(sum(x^2) / H + eps)
+ *   y    = bf16((x * (gain_center + norm_w)) * inv)
+ *   per block of 16 consecutive y:
+ *     sf   = e4m3_rn_satfinite(gs * (max|y| * fl(1/6)))        -> sf[t, block]
+ *     os   = sf != 0 ? 1 / (sf * (1 / gs)) : 0
+ *     code = e2m1 round-to-nearest-even, saturating, of y * os (sign bit iff < 0)
+ *   packed[t, i] = code(2i) | code(2i + 1) << 4
+ *
+ *   x        tp == 1: [M, H] BF16; tp > 1: rank-block [tp, M, H/tp] BF16, the
+ *            layout a dim-0 all-gather of column shards leaves (logical
+ *            x[t, h] is at ((h / (H/tp)) * M + t) * (H/tp) + h % (H/tp))
+ *   norm_w   [H] BF16
+ *   global_scale  device pointer to one FP32 value gs > 0
+ *   packed   [M, H/2] uint8 (out)       sf  [M, H/16] uint8 E4M3 (out, linear)
+ * Supported: H % 16 == 0, H <= 16384, tp >= 1, H % tp == 0, (H/tp) % 16 == 0.
+ */
+int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* norm_w,
+                     float gain_center, float eps, const float* global_scale, uint8_t* packed,
+                     uint8_t* sf, void* stream);
+
+/*
+ * expert_combine -- post-expert RMSNorm of each selected row + weighted sum.
+ *
+ * Source: TensorRT-LLM PR 21356, description, "Post-expert norm and combine"
+ * (weight-first RMSNorm of each selected expert row, the routing weights and
+ * the top-k sum in one pass; a row behind an invalid slot -- -1, or past the
+ * end of the expert output -- is never read); TensorRT-LLM PR 21042 (the
+ * finalize applies the post-expert norm before the weighted top-k sum);
+ * lmdeploy PR 4835 (absent rows marked -1).
+ *
+ * Per token t, acc = +0, then for j = 0 .. k-1 in order, when
+ * 0 <= row_idx[t, j] < num_rows:
+ *   x   = expert_out[row_idx[t, j], :]
+ *   y   = bf16((x * (gain_center + norm_w)) * (1 / sqrt(sum(x^2) / H + eps)))
+ *   acc = fmaf(weights[t, j], y, acc)
+ * out[t, :] = bf16(acc).  Slots outside [0, num_rows) contribute nothing and
+ * their rows are never read; a token without a valid slot outputs zeros.
+ *
+ *   expert_out  [num_rows, H] BF16     row_idx  [T, k] int32
+ *   weights     [T, k] FP32            norm_w   [H] BF16
+ *   out         [T, H] BF16 (out)
+ * Supported: H % 16 == 0, H <= 16384, 1 <= k <= 32, num_rows >= 0.
+ */
+int expert_combine(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                   const float* weights, int T, int k, const uint16_t* norm_w, float gain_center,
+                   float eps, uint16_t* out, void* stream);
+
+/*
+ * residual_join -- gated residual join over the FP32 residual stream, with
+ * the next branch's prenorm optionally fused.
+ *
+ * Source: TensorRT-LLM PR 21356, description, "Gated residual join"
+ * (alpha * residual + beta * rmsnorm(gain * branch) over the FP32 residual
+ * stream, alone or with the next branch's Gemma prenorm; BF16 rounding where
+ * the reference composition rounds).
+ *
+ * Per token t:
+ *   g  = bf16(gain * branch[t, :])
+ *   n  = bf16(g * (1 / sqrt(sum(g^2) / H + eps)))
+ *   residual[t, :] = alpha * residual[t, :] + beta * n        (in place, FP32)
+ *   if next_w != NULL:
+ *     next_prenorm[t, :] = bf16((r * (next_gc + next_w)) * (1 / sqrt(sum(r^2) / H + next_eps)))
+ *     with r the updated residual row.
+ *
+ *   residual [T, H] FP32 (in/out)   branch [T, H] BF16   gain [H] BF16
+ *   next_w   [H] BF16 or NULL        next_prenorm [T, H] BF16 (out) or NULL
+ *   (next_w and next_prenorm are both NULL or both non-NULL)
+ * Supported: H % 16 == 0, H <= 16384.
+ */
+int residual_join(float* residual, const uint16_t* branch, const uint16_t* gain, float alpha,
+                  float beta, float eps, const uint16_t* next_w, float next_gc, float next_eps,
+                  uint16_t* next_prenorm, int T, int H, void* stream);
+
+/*
+ * expert_combine_join -- expert_combine followed by residual_join in one
+ * kernel, the combine's BF16 output serving as the branch.
+ *
+ * Source: as expert_combine and residual_join (the fused decoder boundary of
+ * TensorRT-LLM PR 21356).  Arguments are those of the two calls; `out`
+ * (the combine output) may be NULL when only the residual and the prenorm are
+ * wanted.  Results equal expert_combine then residual_join bit for bit.
+ */
+int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                        const float* weights, int T, int k, const uint16_t* norm_w,
+                        float gain_center, float eps, uint16_t* out, float* residual,
+                        const uint16_t* gain, float alpha, float beta, float join_eps,
+                        const uint16_t* next_w, float next_gc, float next_eps,
+                        uint16_t* next_prenorm, void* stream);
+
+/* Stage ids for moe_boundary_supported(). */
+enum {
+    MB_STAGE_ROUTE = 0,
+    MB_STAGE_NORM_QUANT = 1,
+    MB_STAGE_COMBINE = 2,
+    MB_STAGE_JOIN = 3,
+    MB_STAGE_COMBINE_JOIN = 4,
+};
+
+/*
+ * moe_boundary_supported -- 1 when the stage takes these sizes, else 0 (the
+ * `*_supported` predicates of TensorRT-LLM PR 21356, description).  No side
+ * effects; arguments a stage does not use are ignored.
+ */
+int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* mb_last_error(void);
+
+/*
+ * mb_device_status -- reads and clears the device-side status word of the
+ * current device (synchronous).  Bit 0: a producer's bounded wait for a free
+ * shared-memory slot ran out; bit 1: a drain wait ran out; bit 2: a
+ * consumer's wait for a copied row ran out.  0 means no kernel reported a
+ * timeout since the last call.  Returns -1 (and sets mb_last_error) when the
+ * CUDA runtime fails.
+ */
+int mb_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_BOUNDARY_H */

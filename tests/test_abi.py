@@ -1,0 +1,78 @@
+"""The C-ABI library builds for sm_100a, loads and exports every declared
+symbol, and rejects bad arguments before touching CUDA (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import expert_combine_b200 as eb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_boundary.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("moe_route", "norm_quant_nvfp4", "expert_combine", "residual_join",
+               "expert_combine_join", "moe_boundary_supported", "mb_last_error",
+               "mb_device_status"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = eb.load()
+    for fn in declared_functions():
+        assert hasattr(lib, fn), fn
+
+
+def test_supported_predicate():
+    assert eb.supported(eb.STAGE_ROUTE, 8, 0, 256, 8)
+    assert eb.supported(eb.STAGE_ROUTE, 8, 0, 2560, 22)
+    assert not eb.supported(eb.STAGE_ROUTE, 8, 0, 5000, 8)
+    assert not eb.supported(eb.STAGE_ROUTE, 8, 0, 4, 8)
+    assert not eb.supported(eb.STAGE_ROUTE, 8, 0, 256, 33)
+    assert eb.supported(eb.STAGE_NORM_QUANT, 8, 4096, 0, 0, 4)
+    assert not eb.supported(eb.STAGE_NORM_QUANT, 8, 4096, 0, 0, 3)
+    assert not eb.supported(eb.STAGE_NORM_QUANT, 8, 32768, 0, 0, 1)
+    assert eb.supported(eb.STAGE_COMBINE, 8, 8192, 0, 8)
+    assert not eb.supported(eb.STAGE_COMBINE, 8, 8200, 0, 8)
+    assert eb.supported(eb.STAGE_JOIN, 8, 16384)
+    assert not eb.supported(99, 8, 16)
+
+
+def test_bad_arguments_are_rejected_before_any_launch():
+    lib = eb.load()
+    N = None
+    assert lib.moe_route(N, N, N, -1, 256, 8, N, N, N) == 1
+    assert lib.moe_route(N, N, N, 4, 256, 0, N, N, N) == 2
+    assert lib.moe_route(N, N, N, 0, 256, 8, N, N, N) == 0          # empty: no launch
+    assert lib.moe_route(N, N, N, 4, 256, 8, N, N, N) == 1
+    assert "null" in eb.last_error()
+    odd = ctypes.c_void_p(0x1004)
+    assert lib.moe_route(odd, odd, odd, 4, 256, 8, odd, odd, N) == 1
+    assert "aligned" in eb.last_error()
+    assert lib.norm_quant_nvfp4(N, 4, 100, 1, N, 0.0, 1e-6, N, N, N, N) == 1
+    assert lib.norm_quant_nvfp4(N, 4, 64, 3, N, 0.0, 1e-6, N, N, N, N) == 1
+    assert lib.norm_quant_nvfp4(N, 0, 64, 1, N, 0.0, 1e-6, N, N, N, N) == 0
+    assert lib.expert_combine(N, 10, 64, N, N, 4, 33, N, 0.0, 1e-6, N, N) == 2
+    assert lib.expert_combine(N, -1, 64, N, N, 4, 8, N, 0.0, 1e-6, N, N) == 1
+    assert lib.expert_combine(N, 10, 64, N, N, 0, 8, N, 0.0, 1e-6, N, N) == 0
+    assert lib.residual_join(N, N, N, 1.0, 0.5, 1e-6, N, 1.0, 1e-6, N, 4, 64, N) == 1
+    a = ctypes.c_void_p(0x1000)
+    assert lib.residual_join(a, a, a, 1.0, 0.5, 1e-6, a, 1.0, 1e-6, N, 4, 64, N) == 1
+    assert "both" in eb.last_error()
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        eb.norm_quant_nvfp4(x, 4, torch.zeros(64, dtype=torch.bfloat16), 0.0, 1e-6,
+                            torch.ones(1))

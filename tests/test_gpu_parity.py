@@ -1,0 +1,260 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Small cases are compared in full; the full-size workloads are compared on
+sampled tokens that the oracle computes one by one.  The bar: routing ids and
+NVFP4 codes/scales bit-exact, routing weights within 1e-6 relative, combine and
+prenorm within one BF16 step, the FP32 residual within 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import expert_combine_b200 as eb
+import oracle
+from expert_combine_b200 import synth
+
+from parity import (bf16_ulp_diff, check_combine, check_join_outputs, check_norm_quant,
+                    check_route, oracle_combine, sample_tokens)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ small, in full
+def test_tiny_all_stages(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev)
+    ids, w, nonexact_w = check_route(case)
+    assert nonexact_w == 0
+    check_norm_quant(case)
+    _, nonexact = check_combine(case)
+    assert nonexact == 0
+
+
+@pytest.mark.parametrize("E,k", [(8, 1), (8, 8), (100, 7), (256, 8), (256, 32), (512, 22),
+                                 (2560, 8), (2560, 22), (4096, 32), (33, 32)])
+def test_route_shapes(cuda_dev, E, k):
+    case = synth.make_case("tiny", device=cuda_dev, T=37, E=E, k=k, H=64)
+    check_route(case)
+
+
+def test_route_integer_logits_many_ties(cuda_dev):
+    g = torch.Generator(device=cuda_dev)
+    g.manual_seed(5)
+    for E, k in ((16, 5), (64, 8), (256, 8)):
+        case = synth.make_case("tiny", device=cuda_dev, T=64, E=E, k=k, H=64)
+        case.logits.copy_(torch.randint(-2, 3, case.logits.shape, generator=g, device=cuda_dev))
+        vals = torch.tensor([0.0, 0.125, -0.125], device=cuda_dev)
+        case.bias.copy_(vals[torch.randint(0, 3, (E,), generator=g, device=cuda_dev)])
+        case.logits[case.mask == 0] = float("nan")
+        check_route(case)
+
+
+@pytest.mark.parametrize("H", [16, 48, 272, 1024, 2688, 4096, 8192, 16384])
+@pytest.mark.parametrize("gc", [0.0, 1.0])
+def test_norm_quant_hidden_sizes(cuda_dev, H, gc):
+    case = synth.make_case("tiny", device=cuda_dev, T=19, H=H, gc=gc, join=False)
+    check_norm_quant(case)
+
+
+@pytest.mark.parametrize("H,tp", [(1024, 2), (1024, 4), (4096, 4), (4096, 8), (8192, 8), (768, 3)])
+def test_norm_quant_rank_block(cuda_dev, H, tp):
+    case = synth.make_case("tiny", device=cuda_dev, T=21, H=H, tp=tp, join=False)
+    check_norm_quant(case)
+
+
+def test_norm_quant_zero_scale_and_saturation(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, T=8, H=256, join=False)
+    x = case.x.float()
+    x[0, :16] = 4.0                      # large block; the rest of row 0 tiny negatives
+    x[0, 16:] = -1e-30
+    x[1] = 0.0                           # an all-zero row: inv = 1/sqrt(eps)
+    x[2, 32:48] = 1e4                    # a block far above the global scale's reach
+    case.x.copy_(x.to(torch.bfloat16))
+    case.gs.fill_(1.0)
+    packed, sf, _ = check_norm_quant(case)
+    s = synth.host(sf)
+    assert (s[0, 1:] == 0).all() and (s == 0x7E).any()
+
+
+@pytest.mark.parametrize("H,k", [(16, 1), (48, 3), (1024, 8), (1024, 22), (2688, 8), (4096, 8),
+                                 (8192, 8), (16384, 4), (1024, 32)])
+def test_combine_shapes(cuda_dev, H, k):
+    case = synth.make_case("tiny", device=cuda_dev, T=23, H=H, k=k, E=max(64, k), join=False)
+    check_combine(case)
+
+
+def test_combine_invalid_slots_never_read(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev)
+    idx = case.row_idx
+    assert (idx < 0).sum() >= 2 and (idx >= case.R).sum() == 1
+    out, _ = check_combine(case)
+    assert torch.isfinite(out.float()).all()
+    # every slot invalid for one token: zeros, nothing read
+    case.row_idx[4] = -1
+    case.row_idx[6] = case.R + 1
+    out, _ = check_combine(case)
+    assert (out[4] == 0).all() and (out[6] == 0).all()
+
+
+def test_combine_empty_and_no_rows(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, T=4, H=64, k=2, E=8, join=False)
+    case.row_idx.fill_(-1)
+    out = eb.expert_combine(case.expert_out, 0, case.row_idx, case.comb_wt, case.post_w, 0.0, 1e-6)
+    torch.cuda.synchronize()
+    assert (out == 0).all()
+    z = torch.empty(0, 2, dtype=torch.int32, device=cuda_dev)
+    eb.expert_combine(case.expert_out, case.R, z, torch.empty(0, 2, device=cuda_dev),
+                      case.post_w, 0.0, 1e-6)
+
+
+@pytest.mark.parametrize("H", [64, 1024, 4096, 8192])
+@pytest.mark.parametrize("with_next", [True, False])
+def test_residual_join(cuda_dev, H, with_next):
+    case = synth.make_case("tiny", device=cuda_dev, T=13, H=H, join=True)
+    g = torch.Generator(device=cuda_dev)
+    g.manual_seed(3)
+    branch = torch.randn(case.T, H, generator=g, device=cuda_dev).to(torch.bfloat16)
+    r = case.residual.clone()
+    nw = case.next_w if with_next else None
+    p = eb.residual_join(r, branch, case.gain, case.alpha, case.beta, case.eps, nw, case.next_gc,
+                         case.eps)
+    torch.cuda.synchronize()
+    r_o, p_o = oracle.join(synth.host(case.residual), synth.host(branch), synth.host(case.gain),
+                           case.alpha, case.beta, case.eps,
+                           synth.host(nw) if with_next else None, case.next_gc, case.eps)
+    check_join_outputs(synth.host(r), synth.host(p) if with_next else None, r_o, p_o, case.beta)
+
+
+def test_combine_join_fused_equals_oracle_chain(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, join=True)
+    r = case.residual.clone()
+    out, p = eb.expert_combine_join(case.expert_out, case.R, case.row_idx, case.comb_wt,
+                                    case.post_w, case.post_gc, case.eps, r, case.gain, case.alpha,
+                                    case.beta, case.eps, case.next_w, case.next_gc, case.eps,
+                                    out=torch.empty(case.T, case.H, dtype=torch.bfloat16,
+                                                    device=cuda_dev))
+    torch.cuda.synchronize()
+    branch_o = oracle_combine(case, synth.host(case.comb_wt))
+    assert bf16_ulp_diff(synth.host(out), branch_o).max() <= 1
+    r_o, p_o = oracle.join(synth.host(case.residual), branch_o, synth.host(case.gain), case.alpha,
+                           case.beta, case.eps, synth.host(case.next_w), case.next_gc, case.eps)
+    check_join_outputs(synth.host(r), synth.host(p), r_o, p_o, case.beta)
+
+
+def test_route_then_combine_end_to_end(cuda_dev):
+    """Stage 1's weights feed stage 3, on both sides."""
+    case = synth.make_case("wide_topk", device=cuda_dev, T=300, join=False)
+    ids, w = eb.moe_route(case.logits, case.bias, case.mask, case.k)
+    torch.cuda.synchronize()
+    _, w_o = oracle.route(synth.host(case.logits), synth.host(case.bias), synth.host(case.mask),
+                          case.k)
+    check_combine(case, wt=w, wt_host=w_o)
+
+
+def test_nonblocking_stream_and_determinism(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, T=64, H=2048, join=False)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        p1, s1 = eb.norm_quant_nvfp4(case.x, case.T, case.norm_w, 0.0, case.eps, case.gs)
+        o1 = eb.expert_combine(case.expert_out, case.R, case.row_idx, case.comb_wt, case.post_w,
+                               0.0, case.eps)
+    s.synchronize()
+    p2, s2 = eb.norm_quant_nvfp4(case.x, case.T, case.norm_w, 0.0, case.eps, case.gs)
+    o2 = eb.expert_combine(case.expert_out, case.R, case.row_idx, case.comb_wt, case.post_w, 0.0,
+                           case.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(p1, p2) and torch.equal(s1, s2) and torch.equal(o1, o2)
+    assert eb.device_status() == 0
+
+
+def test_cuda_graph_replay_with_changed_inputs(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, T=32, H=1024, join=False)
+    ids = torch.empty(case.T, case.k, dtype=torch.int32, device=cuda_dev)
+    w = torch.empty(case.T, case.k, dtype=torch.float32, device=cuda_dev)
+    packed = torch.empty(case.T, case.H // 2, dtype=torch.uint8, device=cuda_dev)
+    sf = torch.empty(case.T, case.H // 16, dtype=torch.uint8, device=cuda_dev)
+    out = torch.empty(case.T, case.H, dtype=torch.bfloat16, device=cuda_dev)
+
+    def step():
+        eb.moe_route(case.logits, case.bias, case.mask, case.k, ids, w)
+        eb.norm_quant_nvfp4(case.x, case.T, case.norm_w, 0.0, case.eps, case.gs, packed=packed,
+                            sf=sf)
+        eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, 0.0, case.eps,
+                          out=out)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()                                  # warm-up (first call configures the kernels)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for seed in (11, 12):
+        other = synth.make_case("tiny", device=cuda_dev, T=32, H=1024, join=False, seed=seed)
+        case.logits.copy_(other.logits)
+        case.x.copy_(other.x)
+        case.expert_buf.copy_(other.expert_buf)
+        graph.replay()
+        torch.cuda.synchronize()
+        ids_o, w_o = oracle.route(synth.host(case.logits), synth.host(case.bias),
+                                  synth.host(case.mask), case.k)
+        assert np.array_equal(synth.host(ids), ids_o)
+        p_o, s_o = oracle.norm_quant(synth.host(case.x), case.T, case.H, 1,
+                                     synth.host(case.norm_w), 0.0, case.eps,
+                                     float(synth.host(case.gs)[0]))
+        assert np.array_equal(synth.host(packed), p_o) and np.array_equal(synth.host(sf), s_o)
+        want = oracle_combine(case, w_o)
+        assert bf16_ulp_diff(synth.host(out), want).max() <= 1
+
+
+def test_invalid_arguments_raise(cuda_dev):
+    case = synth.make_case("tiny", device=cuda_dev, T=4, H=64, k=2, E=8, join=False)
+    with pytest.raises(eb.MoEBoundaryError) as ei:
+        eb.moe_route(case.logits, case.bias, case.mask, 0)
+    assert ei.value.status == 2
+    with pytest.raises(eb.MoEBoundaryError):
+        eb.norm_quant_nvfp4(case.x, case.T, case.norm_w, 0.0, 1e-6, case.gs, tp=3)
+    bad = torch.empty(8 * 64 + 8, dtype=torch.bfloat16, device=cuda_dev)[1:][: 4 * 64]
+    with pytest.raises(eb.MoEBoundaryError) as ei:
+        eb.norm_quant_nvfp4(bad, 4, case.norm_w, 0.0, 1e-6, case.gs)
+    assert ei.value.status == 1 and "aligned" in eb.last_error()
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+FULL = ["decode", "prefill", "large_e", "wide_topk"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(cuda_dev, name):
+    case = synth.make_case(name, device=cuda_dev)
+    masked = np.nonzero(synth.host(case.mask) == 0)[0][:4]
+    tokens = sample_tokens(case.T, 48, seed=len(name), must=masked)
+    ids, w, _ = check_route(case, tokens)
+    check_norm_quant(case, tokens)
+    # the combine takes stage 1's weights, as in the benchmark step
+    _, w_o = oracle.route(synth.host(case.logits), synth.host(case.bias), synth.host(case.mask),
+                          case.k) if case.T <= 8192 else (None, None)
+    if w_o is None:
+        wt_host = np.zeros((case.T, case.k), np.float32)
+        tk = torch.as_tensor(tokens, device=cuda_dev)
+        _, w_s = oracle.route(synth.host(case.logits.index_select(0, tk)), synth.host(case.bias),
+                              synth.host(case.mask.index_select(0, tk)), case.k)
+        wt_host[tokens] = w_s
+    else:
+        wt_host = w_o
+    check_combine(case, tokens, wt=w, wt_host=wt_host)
+    if case.residual is not None:
+        r = case.residual.clone()
+        out = torch.empty(case.T, case.H, dtype=torch.bfloat16, device=cuda_dev)
+        _, p = eb.expert_combine_join(case.expert_out, case.R, case.row_idx, w, case.post_w,
+                                      case.post_gc, case.eps, r, case.gain, case.alpha, case.beta,
+                                      case.eps, case.next_w, case.next_gc, case.eps, out=out)
+        torch.cuda.synchronize()
+        branch_o = oracle_combine(case, wt_host, tokens)
+        assert bf16_ulp_diff(synth.host(out)[tokens], branch_o).max() <= 1
+        r_o, p_o = oracle.join(synth.host(case.residual)[tokens], branch_o, synth.host(case.gain),
+                               case.alpha, case.beta, case.eps, synth.host(case.next_w),
+                               case.next_gc, case.eps)
+        check_join_outputs(synth.host(r)[tokens], synth.host(p)[tokens], r_o, p_o, case.beta)
+    assert eb.device_status() == 0
