@@ -66,7 +66,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -229,7 +229,8 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     eb.load()
-    case = synth.make_case(WORKLOAD, device=dev, seed=synth.SEEDS[WORKLOAD] + rank)
+    case = synth.make_case(WORKLOAD, device=dev, seed=synth.SEEDS[WORKLOAD] + rank,
+                           T=args.tokens)
     T, H, E, k = case.T, case.H, case.E, case.k
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
     w = torch.empty(T, k, dtype=torch.float32, device=dev)
@@ -238,18 +239,21 @@ def run_ours(args, world, rank, local):
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    ev = {}
-
-    def step(timed_combine=None):
+    def step(ev=None):
+        # ev: 4 events bracketing the three launches (stage times on this stream)
+        if ev is not None:
+            ev[0].record(stream)
         eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+        if ev is not None:
+            ev[1].record(stream)
         eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
                             sf=sf)
-        if timed_combine is not None:
-            timed_combine[0].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
         eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                           case.eps, out=out)
-        if timed_combine is not None:
-            timed_combine[1].record(stream)
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -257,25 +261,20 @@ def run_ours(args, world, rank, local):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    cmb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
         time.sleep(0.3)
-        # keep the timed region long enough for the clock sampler to see it
         t_wall = time.perf_counter()
         for i in range(args.steps):
-            starts[i].record(stream)
-            step(cmb[i])
-            ends[i].record(stream)
+            step(evs[i])
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     barrier(world)
-    step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    combine_ms = sum(a.elapsed_time(b) for a, b in cmb) / args.steps
+    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
+    combine_ms = stage_ms[2]
     step_ms_max = max_over_ranks(step_ms, world)
     ms_per_step = step_ms_max / args.steps
 
@@ -291,13 +290,14 @@ def run_ours(args, world, rank, local):
     achieved_cmb = cmb_bytes_net / (combine_ms * 1e-3) / 1e9
 
     # end to end through the same calls with host buffers (pinned), copies inside
-    e2e = run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps=max(2, min(args.steps, 5)))
+    e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
+                                           steps=max(2, min(args.steps, 5)))
 
     tokens_per_s = T * world / (ms_per_step * 1e-3)
     result = None
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and T >= 512:
             n_sample = 512
             tokens, ch = host_sample(case, n_sample, seed=2)
             v, cores, reps, med = time_oracle(ch, tokens)
@@ -310,7 +310,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "prefill T=8192 H=8192 E=256 k=8 (route+norm-quant+combine)",
+            "config": {"workload": f"prefill T={T} H=8192 E=256 k=8 (route+norm-quant+combine)",
                        "tokens_per_rank": T, "hidden": H, "experts": E, "top_k": k,
                        "expert_rows": case.R, "valid_tokens": valid_tokens,
                        "valid_slots": valid_slots, "parallelism": f"dp{world}",
@@ -325,6 +325,8 @@ def run_ours(args, world, rank, local):
                          "bytes_per_launch": cmb_bytes_net,
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},
+            "stages_ms": {"route": stage_ms[0], "norm_quant": stage_ms[1],
+                          "combine": stage_ms[2]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,
@@ -378,8 +380,11 @@ def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per rank (default: the workload's 8192); smaller for profiling")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
