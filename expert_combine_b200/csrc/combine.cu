@@ -20,173 +20,191 @@
 // Fused after the combine, `branch` is the BF16 combine output.
 #include "internal.h"
 #include "ring.cuh"
+#include "tmap.h"
 
 namespace mb {
 
-// Join epilogue for one token: this thread holds 16 B branch values of the
-// row (BF16-exact floats in br[]).  Uses two or three team sums.
-template <int B, int TW>
-__device__ __forceinline__ void join_token(const float (&br)[16 * B], int t, int H, int tid, int nvalid,
-                                           const JoinArgs& j, const float (&gain)[16 * B],
-                                           const float (&g2)[16 * B], TeamSum<TW>& team_sum) {
-    float* rrow = j.residual + static_cast<size_t>(t) * H + 16 * B * tid;
-    float r[16 * B];
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (b < nvalid) v = *reinterpret_cast<const float4*>(rrow + 16 * b + 4 * q);
-            r[16 * b + 4 * q + 0] = v.x;
-            r[16 * b + 4 * q + 1] = v.y;
-            r[16 * b + 4 * q + 2] = v.z;
-            r[16 * b + 4 * q + 3] = v.w;
-        }
-    }
-    float gg[16 * B];
-#pragma unroll
-    for (int i = 0; i < 16 * B; ++i) gg[i] = round_bf16(__fmul_rn(gain[i], br[i]));
-    float part[B];
-#pragma unroll
-    for (int b = 0; b < B; ++b) part[b] = block_sumsq16(gg + 16 * b);
-    bool abort;
-    const float ss_g = team_sum(tree_sum_array<B>(part), false, abort);
-    const float inv_g = inv_rms(ss_g, static_cast<float>(H), j.eps);
-#pragma unroll
-    for (int i = 0; i < 16 * B; ++i) {
-        const float n = round_bf16(__fmul_rn(gg[i], inv_g));
-        r[i] = __fadd_rn(__fmul_rn(j.alpha, r[i]), __fmul_rn(j.beta, n));
-    }
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-        if (b < nvalid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<float4*>(rrow + 16 * b + 4 * q) =
-                    make_float4(r[16 * b + 4 * q], r[16 * b + 4 * q + 1], r[16 * b + 4 * q + 2],
-                                r[16 * b + 4 * q + 3]);
-        }
-    }
-    if (j.next_w != nullptr) {
-#pragma unroll
-        for (int b = 0; b < B; ++b) part[b] = (b < nvalid) ? block_sumsq16(r + 16 * b) : 0.0f;
-        const float ss_r = team_sum(tree_sum_array<B>(part), false, abort);
-        const float inv_r = inv_rms(ss_r, static_cast<float>(H), j.next_eps);
-        uint16_t* prow = j.next_prenorm + static_cast<size_t>(t) * H + 16 * B * tid;
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            if (b < nvalid) {
-                uint32_t pk[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int e = 16 * b + 2 * i;
-                    pk[i] = pack_bf16x2(__fmul_rn(__fmul_rn(r[e], g2[e]), inv_r),
-                                        __fmul_rn(__fmul_rn(r[e + 1], g2[e + 1]), inv_r));
-                }
-                *reinterpret_cast<uint4*>(prow + 16 * b) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(prow + 16 * b + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-        }
-    }
-}
-
-template <int B>
-__device__ __forceinline__ void load_gain(const uint16_t* w, float center, int tid, int nvalid,
-                                          float (&g)[16 * B]) {
-#pragma unroll
-    for (int i = 0; i < 16 * B; ++i)
-        g[i] = (w != nullptr && i / 16 < nvalid)
-                   ? __fadd_rn(center, __uint_as_float(static_cast<uint32_t>(w[16 * B * tid + i]) << 16))
-                   : 0.0f;
-}
+struct CombineArgs {
+    const uint16_t* expert_out;
+    int64_t R;
+    int H;
+    const int32_t* row_idx;
+    const float* wt;
+    int T, k;
+    const uint16_t* w;
+    float gc, eps;
+    uint16_t* out;
+    JoinArgs join;
+    int nslot;
+};
 
 __device__ __forceinline__ bool slot_valid(int32_t r, int64_t R) {
     return r >= 0 && static_cast<int64_t>(r) < R;
 }
 
-template <int B, int TW, bool JOIN>
-__global__ void __launch_bounds__(kConsumerThreads + 32, 1)
-    combine_kernel(const uint16_t* __restrict__ expert_out, int64_t R, int H,
-                   const int32_t* __restrict__ row_idx, const float* __restrict__ wt, int T, int k,
-                   const uint16_t* __restrict__ w, float gc, float eps, uint16_t* __restrict__ out,
-                   JoinArgs join, int nslot) {
+__device__ __forceinline__ void load_words32(const uint16_t* p, bool valid0, bool valid1, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if ((c < 2) ? valid0 : valid1) v = *reinterpret_cast<const uint4*>(p + 8 * c);
+        w[4 * c] = v.x;
+        w[4 * c + 1] = v.y;
+        w[4 * c + 2] = v.z;
+        w[4 * c + 3] = v.w;
+    }
+}
+
+// Canonical sum of squares of this thread's 32 FP32 values (pairs r[i] =
+// elements 2i, 2i+1; i < 8 is block 0).
+__device__ __forceinline__ float row32_sumsq_f(const float2 (&r)[16]) {
+    float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 lo = make_float2(r[i].x, r[8 + i].x);
+        const float2 hi = make_float2(r[i].y, r[8 + i].y);
+        a = fma2(lo, lo, a);
+        a = fma2(hi, hi, a);
+    }
+    return a.x + a.y;
+}
+
+// Join epilogue for one token; this thread holds 32 branch values as BF16
+// pair words.  Two or three team sums.
+template <int TW>
+__device__ __forceinline__ void join_token32(const uint32_t (&brw)[16], int t, int H, int tid, int nvalid,
+                                             const JoinArgs& j, TeamSum<TW>& team_sum, bool pow2,
+                                             float rH) {
+    const float fH = static_cast<float>(H);
+    const bool v0 = nvalid > 0, v1 = nvalid > 1;
+    uint32_t gw[16];
+    load_words32(j.gain + 32 * tid, v0, v1, gw);
+    uint32_t gg[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gg[i] = pack_bf16x2_rn(mul2(unpack_bf16x2(gw[i]), unpack_bf16x2(brw[i])));
+    bool abort;
+    const float ss_g = team_sum(row32_sumsq(gg), false, abort);
+    const float inv_g = inv_rms_h(ss_g, fH, rH, pow2, j.eps);
+    const float2 inv_g2 = make_float2(inv_g, inv_g);
+    const float2 alpha2 = make_float2(j.alpha, j.alpha);
+    const float2 beta2 = make_float2(j.beta, j.beta);
+
+    float* rrow = j.residual + static_cast<size_t>(t) * H + 32 * tid;
+    float2 r[16];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if ((c < 4) ? v0 : v1) v = *reinterpret_cast<const float4*>(rrow + 4 * c);
+        r[2 * c] = make_float2(v.x, v.y);
+        r[2 * c + 1] = make_float2(v.z, v.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 n = unpack_bf16x2(pack_bf16x2_rn(mul2(unpack_bf16x2(gg[i]), inv_g2)));
+        r[i] = add2(mul2(alpha2, r[i]), mul2(beta2, n));
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        if ((c < 4) ? v0 : v1)
+            *reinterpret_cast<float4*>(rrow + 4 * c) =
+                make_float4(r[2 * c].x, r[2 * c].y, r[2 * c + 1].x, r[2 * c + 1].y);
+
+    if (j.next_w != nullptr) {
+        const float ss_r = team_sum(row32_sumsq_f(r), false, abort);
+        const float inv_r = inv_rms_h(ss_r, fH, rH, pow2, j.next_eps);
+        const float2 inv_r2 = make_float2(inv_r, inv_r);
+        const float2 gc2 = make_float2(j.next_gc, j.next_gc);
+        uint32_t nw[16];
+        load_words32(j.next_w + 32 * tid, v0, v1, nw);
+        uint32_t pw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            pw[i] = pack_bf16x2_rn(mul2(mul2(r[i], add2(gc2, unpack_bf16x2(nw[i]))), inv_r2));
+        uint16_t* prow = j.next_prenorm + static_cast<size_t>(t) * H + 32 * tid;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if ((c < 2) ? v0 : v1)
+                *reinterpret_cast<uint4*>(prow + 8 * c) =
+                    make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+    }
+}
+
+template <int TW, bool SWZ, bool JOIN>
+__global__ void __launch_bounds__(kConsumerThreads, 1)
+    combine_kernel(const __grid_constant__ CUtensorMap tmap, const CombineArgs a) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int slot_bytes = 2 * H;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_saddr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_saddr + kSlotAlign - 1) & ~uint32_t(kSlotAlign - 1)) - raw_saddr);
+    const int H = a.H;
+    const int nslot = a.nslot;
+    const int slot_bytes = slot_bytes_for(H);
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
     float* red_all = reinterpret_cast<float*>(smem + lay.red_offset());
-    int* flags_all = reinterpret_cast<int*>(red_all + NTEAM * 2 * TW);
+    int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NTEAM * nslot; ++i) {
-            mbar_init(&bars[2 * i], 1);
-            mbar_init(&bars[2 * i + 1], 1);
-        }
+        for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    griddep_wait();     // row indices and weights may come from the previous kernel
+    griddep_launch();
 
+    const int T = a.T, k = a.k;
+    const int64_t R = a.R;
     const int team_stride = gridDim.x * NTEAM;
-
-    if (warp == NTEAM * TW) {
-        // ---------------- producer: lane `team` copies the valid rows of the
-        // team's tokens, in slot order, into the team's ring.
-        if (lane < NTEAM) {
-            const int team = lane;
-            uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
-            uint64_t* tb = bars + static_cast<size_t>(team) * nslot * 2;
-            int fills = 0;
-            bool stop = false;
-            for (int t = blockIdx.x * NTEAM + team; t < T && !stop; t += team_stride) {
-                const int tn = t + team_stride;
-                if (tn < T)
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(row_idx + static_cast<size_t>(tn) * k));
-                const int32_t* ir = row_idx + static_cast<size_t>(t) * k;
-                for (int j = 0; j < k; ++j) {
-                    const int32_t r = __ldg(ir + j);
-                    if (!slot_valid(r, R)) continue;
-                    const int slot = fills % nslot;
-                    const int use = fills / nslot;
-                    if (use > 0 && !mbar_wait_bounded(&tb[2 * slot + 1], (use - 1) & 1, 1u)) {
-                        stop = true;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&tb[2 * slot], static_cast<uint32_t>(slot_bytes));
-                    bulk_g2s(ring + static_cast<size_t>(slot) * slot_bytes,
-                             expert_out + static_cast<size_t>(r) * H, static_cast<uint32_t>(slot_bytes),
-                             &tb[2 * slot]);
-                    ++fills;
-                }
-            }
-            for (int f = fills > nslot ? fills - nslot : 0; f < fills; ++f)
-                mbar_wait_bounded(&tb[2 * (f % nslot)], (f / nslot) & 1, 2u);
-        }
-        return;
-    }
-
-    // ---------------- consumers
     const int team = warp / TW;
     const int warp_in_team = warp % TW;
     const int tid = warp_in_team * 32 + lane;
     const int nblocks = H / 16;
-    int nvalid = nblocks - tid * B;
-    nvalid = nvalid < 0 ? 0 : (nvalid > B ? B : nvalid);
-    const uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
-    uint64_t* tb = bars + static_cast<size_t>(team) * nslot * 2;
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, flags_all + team * 2 * TW, 1 + team, warp_in_team,
-                         lane, 0};
+    int nvalid = nblocks - 2 * tid;
+    nvalid = nvalid < 0 ? 0 : (nvalid > 2 ? 2 : nvalid);
+    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
+    const uint32_t ring_saddr = smem_addr(ring);
+    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
+    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
 
-    float g[16 * B];
-    load_gain<B>(w, gc, tid, nvalid, g);
-    float gain[16 * B], g2[16 * B];
-    if constexpr (JOIN) {
-        load_gain<B>(join.gain, 0.0f, tid, nvalid, gain);
-        load_gain<B>(join.next_w, join.next_gc, tid, nvalid, g2);
+    // ---- the leader's copy cursor over (token, slot): valid rows in order
+    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
+    auto issue = [&]() {
+        int ct = cur->ct, cj = cur->cj;
+        while (ct < T) {
+            const int32_t r = __ldg(a.row_idx + static_cast<size_t>(ct) * k + cj);
+            if (++cj == k) {
+                cj = 0;
+                ct += team_stride;
+                if (ct + team_stride < T)
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.row_idx + static_cast<size_t>(ct + team_stride) * k));
+            }
+            if (!slot_valid(r, R)) continue;
+            const int ws = cur->wslot;
+            mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
+            uint8_t* dst = ring + static_cast<size_t>(ws) * slot_bytes;
+            if constexpr (SWZ)
+                tma_load_2d(smem_addr(dst), &tmap, 0, r * (H / 64), &tb[ws]);
+            else
+                bulk_g2s(dst, a.expert_out + static_cast<size_t>(r) * H, 2u * static_cast<uint32_t>(H), &tb[ws]);
+            cur->issued += 1;
+            cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
+            break;
+        }
+        cur->ct = ct;
+        cur->cj = cj;
+    };
+    if (tid == 0) {
+        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < nslot; ++i) issue();
     }
+
+    float2 g[16];
+    load_gain32(a.w, a.gc, tid, nvalid, g);
     const float fH = static_cast<float>(H);
+    const bool pow2 = (H & (H - 1)) == 0;
+    const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
 
     // slot indices and weights of the token, one slot per lane (k <= 32),
     // loaded one token ahead
@@ -194,199 +212,199 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1)
     int32_t my_r = -1;
     float my_w = 0.0f;
     if (t < T && lane < k) {
-        my_r = __ldg(row_idx + static_cast<size_t>(t) * k + lane);
-        my_w = __ldg(wt + static_cast<size_t>(t) * k + lane);
+        my_r = __ldg(a.row_idx + static_cast<size_t>(t) * k + lane);
+        my_w = __ldg(a.wt + static_cast<size_t>(t) * k + lane);
     }
-    int fills = 0;
+    int slot = 0, phase = 0;
     bool aborted = false;
     for (; t < T; t += team_stride) {
         const int32_t cur_r = my_r;
         const float cur_w = my_w;
         const int tn = t + team_stride;
         if (tn < T && lane < k) {
-            my_r = __ldg(row_idx + static_cast<size_t>(tn) * k + lane);
-            my_w = __ldg(wt + static_cast<size_t>(tn) * k + lane);
+            my_r = __ldg(a.row_idx + static_cast<size_t>(tn) * k + lane);
+            my_w = __ldg(a.wt + static_cast<size_t>(tn) * k + lane);
         }
-        float acc[16 * B];
+        float2 acc[16];
 #pragma unroll
-        for (int i = 0; i < 16 * B; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
 
         for (int j = 0; j < k; ++j) {
             const int32_t r = __shfl_sync(0xffffffffu, cur_r, j);
             if (!slot_valid(r, R)) continue;
             const float wj = __shfl_sync(0xffffffffu, cur_w, j);
-            const int slot = fills % nslot;
-            const bool ok = mbar_wait_bounded(&tb[2 * slot], (fills / nslot) & 1, 4u);
-            uint32_t wv[8 * B];
+            const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
+            uint32_t wv[16];
             if (ok) {
-                read_slot_blocks<B>(ring + static_cast<size_t>(slot) * slot_bytes, tid, nvalid, wv);
+                read_row32<SWZ>(ring_saddr + static_cast<uint32_t>(slot * slot_bytes), tid, nvalid, wv);
             } else {
 #pragma unroll
-                for (int i = 0; i < 8 * B; ++i) wv[i] = 0u;
+                for (int i = 0; i < 16; ++i) wv[i] = 0u;
             }
-            float xv[16 * B];
-#pragma unroll
-            for (int i = 0; i < 8 * B; ++i) {
-                xv[2 * i] = bf16_lo(wv[i]);
-                xv[2 * i + 1] = bf16_hi(wv[i]);
-            }
-            float part[B];
-#pragma unroll
-            for (int b = 0; b < B; ++b) part[b] = block_sumsq16(xv + 16 * b);
             bool abort;
-            const float ss = team_sum(tree_sum_array<B>(part), !ok, abort);
+            const float ss = team_sum(row32_sumsq(wv), !ok, abort);
             if (abort) {
                 aborted = true;
                 break;
             }
-            if (tid == 0) mbar_arrive(&tb[2 * slot + 1]);
-            ++fills;
-            const float inv = inv_rms(ss, fH, eps);
+            if (tid == 0) {   // the whole team has read this slot: refill it
+                cur->consumed += 1;
+                fence_proxy_async_smem();
+                issue();
+            }
+            if (++slot == nslot) {
+                slot = 0;
+                phase ^= 1;
+            }
+            const float inv = inv_rms_h(ss, fH, rH, pow2, a.eps);
+            const float2 inv2 = make_float2(inv, inv);
+            const float2 w2 = make_float2(wj, wj);
 #pragma unroll
-            for (int i = 0; i < 16 * B; ++i)
-                acc[i] = fmaf(wj, round_bf16(__fmul_rn(__fmul_rn(xv[i], g[i]), inv)), acc[i]);
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t y = pack_bf16x2_rn(mul2(mul2(unpack_bf16x2(wv[i]), g[i]), inv2));
+                acc[i] = fma2(w2, unpack_bf16x2(y), acc[i]);
+            }
         }
         if (aborted) break;
 
-        float br[16 * B];
+        uint32_t brw[16];
 #pragma unroll
-        for (int i = 0; i < 16 * B; ++i) br[i] = round_bf16(acc[i]);
-        if (out != nullptr) {
-            uint16_t* orow = out + static_cast<size_t>(t) * H + 16 * B * tid;
+        for (int i = 0; i < 16; ++i) brw[i] = pack_bf16x2_rn(acc[i]);
+        if (a.out != nullptr) {
+            uint16_t* orow = a.out + static_cast<size_t>(t) * H + 32 * tid;
 #pragma unroll
-            for (int b = 0; b < B; ++b) {
-                if (b < nvalid) {
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(br[16 * b + 2 * i], br[16 * b + 2 * i + 1]);
-                    *reinterpret_cast<uint4*>(orow + 16 * b) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4*>(orow + 16 * b + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                }
-            }
+            for (int c = 0; c < 4; ++c)
+                if (c / 2 < nvalid)
+                    *reinterpret_cast<uint4*>(orow + 8 * c) =
+                        make_uint4(brw[4 * c], brw[4 * c + 1], brw[4 * c + 2], brw[4 * c + 3]);
         }
-        if constexpr (JOIN) join_token<B, TW>(br, t, H, tid, nvalid, join, gain, g2, team_sum);
+        if constexpr (JOIN) join_token32<TW>(brw, t, H, tid, nvalid, a.join, team_sum, pow2, rH);
     }
+    // copies still in flight (only after an abort) land before the CTA exits
+    if (tid == 0)
+        for (int f = cur->consumed; f < cur->issued; ++f)
+            mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
 }
 
 // Standalone gated residual join: the branch comes from global memory.
-template <int B, int TW>
+template <int TW>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     residual_join_kernel(const uint16_t* __restrict__ branch, int T, int H, JoinArgs join) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    __shared__ float red_all[NTEAM * 2 * TW];
-    __shared__ int flags_all[NTEAM * 2 * TW];
+    __shared__ __align__(16) float red_all[NTEAM * 2 * TW];
+    __shared__ int abort_all[NTEAM * 4];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int team = warp / TW;
     const int warp_in_team = warp % TW;
     const int tid = warp_in_team * 32 + lane;
     const int nblocks = H / 16;
-    int nvalid = nblocks - tid * B;
-    nvalid = nvalid < 0 ? 0 : (nvalid > B ? B : nvalid);
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, flags_all + team * 2 * TW, 1 + team, warp_in_team,
-                         lane, 0};
-    float gain[16 * B], g2[16 * B];
-    load_gain<B>(join.gain, 0.0f, tid, nvalid, gain);
-    load_gain<B>(join.next_w, join.next_gc, tid, nvalid, g2);
+    int nvalid = nblocks - 2 * tid;
+    nvalid = nvalid < 0 ? 0 : (nvalid > 2 ? 2 : nvalid);
+    if (threadIdx.x < NTEAM) abort_all[4 * threadIdx.x] = 0;
+    __syncthreads();
+    griddep_wait();
+    griddep_launch();
+    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
+    const bool pow2 = (H & (H - 1)) == 0;
+    const float rH = pow2 ? __frcp_rn(static_cast<float>(H)) : 0.0f;
     for (int t = blockIdx.x * NTEAM + team; t < T; t += gridDim.x * NTEAM) {
-        const uint16_t* brow = branch + static_cast<size_t>(t) * H + 16 * B * tid;
-        float br[16 * B];
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-            if (b < nvalid) {
-                lo = ld_nc_v4(brow + 16 * b);
-                hi = ld_nc_v4(brow + 16 * b + 8);
-            }
-            const uint32_t v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                br[16 * b + 2 * i] = bf16_lo(v[i]);
-                br[16 * b + 2 * i + 1] = bf16_hi(v[i]);
-            }
-        }
-        join_token<B, TW>(br, t, H, tid, nvalid, join, gain, g2, team_sum);
+        uint32_t brw[16];
+        load_words32(branch + static_cast<size_t>(t) * H + 32 * tid, nvalid > 0, nvalid > 1, brw);
+        join_token32<TW>(brw, t, H, tid, nvalid, join, team_sum, pow2, rH);
     }
 }
 
 namespace {
 
-template <int B, int TW>
-cudaError_t launch_cb(const uint16_t* expert_out, int64_t R, int H, const int32_t* row_idx, const float* wt,
-                      int T, int k, const uint16_t* w, float gc, float eps, uint16_t* out,
-                      const JoinArgs& join, cudaStream_t s) {
+cudaLaunchConfig_t pdl_config(int grid, int block, size_t smem, cudaStream_t s, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+template <int TW, bool SWZ, bool JOIN>
+cudaError_t launch_cb(const CUtensorMap& tmap, const CombineArgs& args, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    const int slot_bytes = 2 * H;
+    const int slot_bytes = slot_bytes_for(args.H);
     int nslot = kRingBytes / (NTEAM * slot_bytes);
     if (nslot > 16) nslot = 16;
     if (nslot < 2) return cudaErrorInvalidConfiguration;
+    CombineArgs a = args;
+    a.nslot = nslot;
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     const size_t smem = lay.total_bytes();
-    int grid = (T + NTEAM - 1) / NTEAM;
+    auto kern = combine_kernel<TW, SWZ, JOIN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int grid = (a.T + NTEAM - 1) / NTEAM;
     const int cap = device_info().sm_count;
     if (grid > cap) grid = cap;
-    if (join.residual != nullptr) {
-        auto kern = combine_kernel<B, TW, true>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kConsumerThreads + 32, smem, s>>>(expert_out, R, H, row_idx, wt, T, k, w, gc, eps,
-                                                        out, join, nslot);
-    } else {
-        auto kern = combine_kernel<B, TW, false>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kConsumerThreads + 32, smem, s>>>(expert_out, R, H, row_idx, wt, T, k, w, gc, eps,
-                                                        out, join, nslot);
-    }
-    return cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pdl_config(grid, kConsumerThreads, smem, s, attr);
+    return cudaLaunchKernelEx(&cfg, kern, tmap, a);
 }
 
-template <int B, int TW>
+template <bool SWZ, bool JOIN>
+cudaError_t launch_cb_tw(int TW, const CUtensorMap& tmap, const CombineArgs& a, cudaStream_t s) {
+    switch (TW) {
+        case 1: return launch_cb<1, SWZ, JOIN>(tmap, a, s);
+        case 2: return launch_cb<2, SWZ, JOIN>(tmap, a, s);
+        case 4: return launch_cb<4, SWZ, JOIN>(tmap, a, s);
+        case 8: return launch_cb<8, SWZ, JOIN>(tmap, a, s);
+        case 16: return launch_cb<16, SWZ, JOIN>(tmap, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int TW>
 cudaError_t launch_rj(const uint16_t* branch, int T, int H, const JoinArgs& join, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
     int grid = (T + NTEAM - 1) / NTEAM;
     const int cap = device_info().sm_count * 2;
     if (grid > cap) grid = cap;
-    residual_join_kernel<B, TW><<<grid, kConsumerThreads, 0, s>>>(branch, T, H, join);
-    return cudaGetLastError();
-}
-
-void team_shape(int H, int& B, int& TW) {
-    const int nblocks = H / 16;
-    B = nblocks <= 512 ? 1 : 2;
-    const int per = (nblocks + B - 1) / B;
-    int P = 32;
-    while (P < per) P <<= 1;
-    TW = P / 32;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pdl_config(grid, kConsumerThreads, 0, s, attr);
+    return cudaLaunchKernelEx(&cfg, residual_join_kernel<TW>, branch, T, H, join);
 }
 
 }  // namespace
 
+int team_warps(int H);   // norm_quant.cu
+
 cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const int32_t* row_idx,
                            const float* wt, int T, int k, const uint16_t* w, float gc, float eps,
                            uint16_t* out, const JoinArgs& join, cudaStream_t s) {
-    int B, TW;
-    team_shape(H, B, TW);
-#define MB_CB(Bv, TWv) \
-    if (B == Bv && TW == TWv) return launch_cb<Bv, TWv>(expert_out, R, H, row_idx, wt, T, k, w, gc, eps, out, join, s);
-    MB_CB(1, 1) MB_CB(1, 2) MB_CB(1, 4) MB_CB(1, 8) MB_CB(1, 16)
-    MB_CB(2, 16)
-#undef MB_CB
-    return cudaErrorInvalidValue;
+    const CombineArgs a{expert_out, R, H, row_idx, wt, T, k, w, gc, eps, out, join, 0};
+    const int TW = team_warps(H);
+    const bool fused = join.residual != nullptr;
+    CUtensorMap tmap;
+    const bool swz = H % 64 == 0 && R > 0 && static_cast<uint64_t>(R) * (H / 64) < (1ull << 31) &&
+                     encode_line_map(&tmap, expert_out, static_cast<uint64_t>(R) * (H / 64),
+                                     static_cast<uint32_t>(H / 64));
+    if (!swz) std::memset(&tmap, 0, sizeof(tmap));
+    if (swz) return fused ? launch_cb_tw<true, true>(TW, tmap, a, s) : launch_cb_tw<true, false>(TW, tmap, a, s);
+    return fused ? launch_cb_tw<false, true>(TW, tmap, a, s) : launch_cb_tw<false, false>(TW, tmap, a, s);
 }
 
 cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,
                                  cudaStream_t s) {
-    int B, TW;
-    team_shape(H, B, TW);
-#define MB_RJ(Bv, TWv) \
-    if (B == Bv && TW == TWv) return launch_rj<Bv, TWv>(branch, T, H, join, s);
-    MB_RJ(1, 1) MB_RJ(1, 2) MB_RJ(1, 4) MB_RJ(1, 8) MB_RJ(1, 16)
-    MB_RJ(2, 16)
-#undef MB_RJ
-    return cudaErrorInvalidValue;
+    switch (team_warps(H)) {
+        case 1: return launch_rj<1>(branch, T, H, join, s);
+        case 2: return launch_rj<2>(branch, T, H, join, s);
+        case 4: return launch_rj<4>(branch, T, H, join, s);
+        case 8: return launch_rj<8>(branch, T, H, join, s);
+        case 16: return launch_rj<16>(branch, T, H, join, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace mb

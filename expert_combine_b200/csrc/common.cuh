@@ -191,12 +191,9 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
 }
 
 // Eight E2M1 codes packed in a 32-bit word, v[0] in the lowest nibble
-// (round-to-nearest-even on the E2M1 grid, saturating).  A -0 input is made
-// +0 first, so only strictly negative values carry the sign bit.
+// (round-to-nearest-even on the E2M1 grid, saturating).  The caller passes no
+// -0 (a -0 would come back with the sign bit set).
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
-    float z[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) z[i] = __fadd_rn(v[i], 0.0f);
     uint32_t r;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -205,8 +202,83 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
         "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(r)
-        : "f"(z[0]), "f"(z[1]), "f"(z[2]), "f"(z[3]), "f"(z[4]), "f"(z[5]), "f"(z[6]), "f"(z[7]));
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return r;
 }
+
+}  // namespace mb
+
+// ------------------------------------------------------------------ paired FP32 (sm_100 f32x2)
+// Two independent IEEE binary32 operations per instruction; each lane of the
+// pair is rounded exactly like the scalar operation.
+namespace mb {
+
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+    return r;
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t r) {
+    float2 a;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+    return a;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(d);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+    return bits_f2(d);
+}
+// BF16 pair word -> two floats (exact).
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// Two floats -> BF16 pair word, round to nearest even, x in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float2 v) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+// Largest magnitude of the two BF16 halves of a and b, per half (signs are
+// not meaningful in the result; only the magnitudes are used).
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// 2-D tiled TMA load global -> shared (no multicast), completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// its later async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 }  // namespace mb

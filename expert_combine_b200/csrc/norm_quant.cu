@@ -11,185 +11,237 @@
 //                     code = e2m1_rn_satfinite(y * os), -0 carries no sign
 //   packed[t, i] = code(2i) | code(2i + 1) << 4,  sf[t, b] linear [M, H/16]
 // The input row is read either contiguous ([M, H]) or from the rank-block
-// layout [tp, M, H/tp] (tp bulk copies per row into one slot).
+// layout [tp, M, H/tp] (tp copies per row into one slot).
 #include "internal.h"
 #include "ring.cuh"
+#include "tmap.h"
 
 namespace mb {
 
-template <int B, int TW>
-__global__ void __launch_bounds__(kConsumerThreads + 32, 1)
-    norm_quant_kernel(const uint16_t* __restrict__ x, int M, int H, int tp,
-                      const uint16_t* __restrict__ w, float gc, float eps,
-                      const float* __restrict__ gs_ptr, uint8_t* __restrict__ packed,
-                      uint8_t* __restrict__ sf_out, int nslot) {
+struct NormQuantArgs {
+    const uint16_t* x;
+    int M, H, tp;
+    const uint16_t* w;
+    float gc, eps;
+    const float* gs;
+    uint8_t* packed;
+    uint8_t* sf;
+    int nslot;
+};
+
+template <int TW, bool SWZ>
+__global__ void __launch_bounds__(kConsumerThreads, 1)
+    norm_quant_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int slot_bytes = 2 * H;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_saddr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_saddr + kSlotAlign - 1) & ~uint32_t(kSlotAlign - 1)) - raw_saddr);
+    const int H = a.H;
+    const int nslot = a.nslot;
+    const int slot_bytes = slot_bytes_for(H);
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
     float* red_all = reinterpret_cast<float*>(smem + lay.red_offset());
-    int* flags_all = reinterpret_cast<int*>(red_all + NTEAM * 2 * TW);
+    int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NTEAM * nslot; ++i) {
-            mbar_init(&bars[2 * i], 1);       // full: producer's arrive + bytes
-            mbar_init(&bars[2 * i + 1], 1);   // empty: one consumer arrive
-        }
+        for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);   // one arrive + the bytes
+        for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    griddep_wait();     // inputs may come from the previous kernel on the stream
+    griddep_launch();   // the next kernel may start its prologue as CTAs retire
 
+    const int M = a.M;
     const int team_stride = gridDim.x * NTEAM;
-
-    if (warp == NTEAM * TW) {
-        // ---------------- producer: lane `team` feeds that team's ring
-        if (lane < NTEAM) {
-            const int team = lane;
-            uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
-            uint64_t* tb = bars + static_cast<size_t>(team) * nslot * 2;
-            const int hs = H / tp;
-            const uint32_t seg_bytes = 2u * static_cast<uint32_t>(hs);
-            int fills = 0;
-            for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride) {
-                const int slot = fills % nslot;
-                const int use = fills / nslot;
-                if (use > 0 && !mbar_wait_bounded(&tb[2 * slot + 1], (use - 1) & 1, 1u)) break;
-                mbar_arrive_expect_tx(&tb[2 * slot], static_cast<uint32_t>(slot_bytes));
-                uint8_t* dst = ring + static_cast<size_t>(slot) * slot_bytes;
-                for (int s = 0; s < tp; ++s)
-                    bulk_g2s(dst + static_cast<size_t>(s) * seg_bytes,
-                             x + (static_cast<size_t>(s) * M + t) * hs, seg_bytes, &tb[2 * slot]);
-                ++fills;
-            }
-            // drain: every issued copy has landed before the CTA exits
-            for (int f = fills > nslot ? fills - nslot : 0; f < fills; ++f)
-                mbar_wait_bounded(&tb[2 * (f % nslot)], (f / nslot) & 1, 2u);
-        }
-        return;
-    }
-
-    // ---------------- consumers
     const int team = warp / TW;
     const int warp_in_team = warp % TW;
     const int tid = warp_in_team * 32 + lane;
     const int nblocks = H / 16;
-    int nvalid = nblocks - tid * B;
-    nvalid = nvalid < 0 ? 0 : (nvalid > B ? B : nvalid);
-    const uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
-    uint64_t* tb = bars + static_cast<size_t>(team) * nslot * 2;
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, flags_all + team * 2 * TW, 1 + team, warp_in_team,
-                         lane, 0};
+    int nvalid = nblocks - 2 * tid;
+    nvalid = nvalid < 0 ? 0 : (nvalid > 2 ? 2 : nvalid);
+    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
+    const uint32_t ring_saddr = smem_addr(ring);
+    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
+    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
 
-    float g[16 * B];
-#pragma unroll
-    for (int i = 0; i < 16 * B; ++i) {
-        const int h = 16 * B * tid + i;
-        g[i] = (i / 16 < nvalid) ? __fadd_rn(gc, __uint_as_float(static_cast<uint32_t>(w[h]) << 16)) : 0.0f;
+    // ---- the leader's copy cursor: one row (tp segments) per token
+    const int hs = H / a.tp;
+    const uint32_t seg_bytes = 2u * static_cast<uint32_t>(hs);
+    const int seg_lines = hs / 64;
+    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
+    auto issue = [&]() {
+        const int nt = cur->ct;
+        if (nt >= M) return;
+        const int ws = cur->wslot;
+        mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
+        uint8_t* dst = ring + static_cast<size_t>(ws) * slot_bytes;
+        for (int s = 0; s < a.tp; ++s) {
+            if constexpr (SWZ)
+                tma_load_2d(smem_addr(dst + static_cast<size_t>(s) * seg_bytes), &tmap, 0,
+                            (s * M + nt) * seg_lines, &tb[ws]);
+            else
+                bulk_g2s(dst + static_cast<size_t>(s) * seg_bytes,
+                         a.x + (static_cast<size_t>(s) * M + nt) * hs, seg_bytes, &tb[ws]);
+        }
+        cur->ct = nt + team_stride;
+        cur->issued += 1;
+        cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
+    };
+    if (tid == 0) {
+        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < nslot; ++i) issue();
     }
-    const float gs = __ldg(gs_ptr);
+
+    float2 g[16];
+    load_gain32(a.w, a.gc, tid, nvalid, g);
+    const float gs = __ldg(a.gs);
     const float rgs = __frcp_rn(gs);
     constexpr float kR6 = (float)(1.0 / 6.0);
     const float fH = static_cast<float>(H);
+    const bool pow2 = (H & (H - 1)) == 0;
+    const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
+    const float2 zero2 = make_float2(0.0f, 0.0f);
 
-    int fills = 0;
+    int slot = 0, phase = 0;
     for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride) {
-        const int slot = fills % nslot;
-        const bool ok = mbar_wait_bounded(&tb[2 * slot], (fills / nslot) & 1, 4u);
-        uint32_t wv[8 * B];
+        const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
+        uint32_t wv[16];
         if (ok) {
-            read_slot_blocks<B>(ring + static_cast<size_t>(slot) * slot_bytes, tid, nvalid, wv);
+            read_row32<SWZ>(ring_saddr + static_cast<uint32_t>(slot * slot_bytes), tid, nvalid, wv);
         } else {
 #pragma unroll
-            for (int i = 0; i < 8 * B; ++i) wv[i] = 0u;
+            for (int i = 0; i < 16; ++i) wv[i] = 0u;
         }
-        float xv[16 * B];
-#pragma unroll
-        for (int i = 0; i < 8 * B; ++i) {
-            xv[2 * i] = bf16_lo(wv[i]);
-            xv[2 * i + 1] = bf16_hi(wv[i]);
-        }
-        float part[B];
-#pragma unroll
-        for (int b = 0; b < B; ++b) part[b] = block_sumsq16(xv + 16 * b);
         bool abort;
-        const float ss = team_sum(tree_sum_array<B>(part), !ok, abort);
+        const float ss = team_sum(row32_sumsq(wv), !ok, abort);
         if (abort) break;
-        if (tid == 0) mbar_arrive(&tb[2 * slot + 1]);
-        ++fills;
+        if (tid == 0) {   // the whole team has read this slot: refill it
+            cur->consumed += 1;
+            fence_proxy_async_smem();
+            issue();
+        }
+        if (++slot == nslot) {
+            slot = 0;
+            phase ^= 1;
+        }
 
-        const float inv = inv_rms(ss, fH, eps);
+        const float inv = inv_rms_h(ss, fH, rH, pow2, a.eps);
+        const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
+        for (int b = 0; b < 2; ++b) {
             if (b < nvalid) {
-                float y[16];
-                float amax = 0.0f;
+                uint32_t yw[8];
+                uint32_t m = 0u;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    y[i] = round_bf16(__fmul_rn(__fmul_rn(xv[16 * b + i], g[16 * b + i]), inv));
-                    amax = fmaxf(amax, fabsf(y[i]));
+                for (int i = 0; i < 8; ++i) {
+                    const float2 t2 = mul2(mul2(unpack_bf16x2(wv[8 * b + i]), g[8 * b + i]), inv2);
+                    yw[i] = pack_bf16x2_rn(t2);
+                    m = maxabs_bf16x2(m, yw[i]);
                 }
+                const float2 mf = unpack_bf16x2(m & 0x7fff7fffu);
+                const float amax = fmaxf(mf.x, mf.y);
                 const uint32_t sfc = cvt_e4m3_satfinite(__fmul_rn(gs, __fmul_rn(amax, kR6)));
                 const float sf_f = e4m3_to_f32(sfc);
                 const float os = (sf_f != 0.0f) ? __frcp_rn(__fmul_rn(sf_f, rgs)) : 0.0f;
+                const float2 os2 = make_float2(os, os);
                 float q[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(y[i], os);
+                for (int i = 0; i < 8; ++i) {
+                    // + 0 turns a -0 product into +0 (no sign bit for -0)
+                    const float2 q2 = add2(mul2(unpack_bf16x2(yw[i]), os2), zero2);
+                    q[2 * i] = q2.x;
+                    q[2 * i + 1] = q2.y;
+                }
                 uint2 codes;
                 codes.x = cvt_e2m1x8(q);
                 codes.y = cvt_e2m1x8(q + 8);
-                const int gb = tid * B + b;
-                *reinterpret_cast<uint2*>(packed + static_cast<size_t>(t) * (H / 2) + 8 * gb) = codes;
-                sf_out[static_cast<size_t>(t) * nblocks + gb] = static_cast<uint8_t>(sfc);
+                const int gb = 2 * tid + b;
+                *reinterpret_cast<uint2*>(a.packed + static_cast<size_t>(t) * (H / 2) + 8 * gb) = codes;
+                a.sf[static_cast<size_t>(t) * nblocks + gb] = static_cast<uint8_t>(sfc);
             }
         }
     }
+    // copies still in flight (only after an abort) land before the CTA exits
+    if (tid == 0)
+        for (int f = cur->consumed; f < cur->issued; ++f)
+            mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
 }
 
 namespace {
 
-template <int B, int TW>
-cudaError_t launch_nq(const uint16_t* x, int M, int H, int tp, const uint16_t* w, float gc, float eps,
-                      const float* gs, uint8_t* packed, uint8_t* sf, cudaStream_t s) {
+template <int TW, bool SWZ>
+cudaError_t launch_nq(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    const int slot_bytes = 2 * H;
+    const int slot_bytes = slot_bytes_for(args.H);
     int nslot = kRingBytes / (NTEAM * slot_bytes);
     if (nslot > 16) nslot = 16;
     if (nslot < 2) return cudaErrorInvalidConfiguration;
+    NormQuantArgs a = args;
+    a.nslot = nslot;
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     const size_t smem = lay.total_bytes();
-    auto kern = norm_quant_kernel<B, TW>;
+    auto kern = norm_quant_kernel<TW, SWZ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    int grid = (M + NTEAM - 1) / NTEAM;
+    int grid = (a.M + NTEAM - 1) / NTEAM;
     const int cap = device_info().sm_count;
     if (grid > cap) grid = cap;
-    kern<<<grid, kConsumerThreads + 32, smem, s>>>(x, M, H, tp, w, gc, eps, gs, packed, sf, nslot);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kConsumerThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, a);
+}
+
+template <bool SWZ>
+cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
+    switch (TW) {
+        case 1: return launch_nq<1, SWZ>(tmap, a, s);
+        case 2: return launch_nq<2, SWZ>(tmap, a, s);
+        case 4: return launch_nq<4, SWZ>(tmap, a, s);
+        case 8: return launch_nq<8, SWZ>(tmap, a, s);
+        case 16: return launch_nq<16, SWZ>(tmap, a, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
-// Team width from the row size: B blocks per thread, P = next_pow2(blocks/B)
-// threads per team (at least one warp).
+// Warps per team: 32 elements per thread, P = next_pow2(H / 32) threads (at
+// least one warp).
+int team_warps(int H) {
+    const int nblocks = H / 16;
+    const int per = (nblocks + 1) / 2;
+    int P = 32;
+    while (P < per) P <<= 1;
+    return P / 32;
+}
+
 cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uint16_t* w, float gc,
                               float eps, const float* gs, uint8_t* packed, uint8_t* sf,
                               cudaStream_t s) {
-    const int nblocks = H / 16;
-    const int B = nblocks <= 512 ? 1 : 2;
-    int per = (nblocks + B - 1) / B;
-    int P = 32;
-    while (P < per) P <<= 1;
-    const int TW = P / 32;
-#define MB_NQ(Bv, TWv) \
-    if (B == Bv && TW == TWv) return launch_nq<Bv, TWv>(x, M, H, tp, w, gc, eps, gs, packed, sf, s);
-    MB_NQ(1, 1) MB_NQ(1, 2) MB_NQ(1, 4) MB_NQ(1, 8) MB_NQ(1, 16)
-    MB_NQ(2, 16)
-#undef MB_NQ
-    return cudaErrorInvalidValue;
+    const NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
+    const int hs = H / tp;
+    // the tensor path needs 64-element lines and each segment on a swizzle atom
+    const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
+                     static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
+    CUtensorMap tmap;
+    if (swz && encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64),
+                               static_cast<uint32_t>(hs / 64)))
+        return launch_nq_tw<true>(team_warps(H), tmap, a, s);
+    std::memset(&tmap, 0, sizeof(tmap));
+    return launch_nq_tw<false>(team_warps(H), tmap, a, s);
 }
 
 }  // namespace mb

@@ -1,58 +1,86 @@
 // ring.cuh -- the row-streaming skeleton shared by the norm-quant and the
 // post-expert combine kernels.
 //
-// A persistent CTA holds NTEAM "teams" of TW consumer warps plus one producer
-// warp.  Each team owns a ring of NSLOT shared-memory row slots; lane `team`
-// of the producer warp fills the team's slots with 1-D bulk copies
-// (cp.async.bulk, completion counted on the slot's "full" mbarrier) while the
-// team consumes them in order and hands each slot back on its "empty"
-// mbarrier.  Rows therefore stream through shared memory with no registers
-// held in flight, and the producer runs up to NSLOT rows ahead.
+// A persistent CTA of 16 warps is split into NTEAM "teams" of TW warps.  Each
+// team owns a ring of NSLOT shared-memory row slots, filled by TMA copies whose
+// completion is counted on the slot's "full" mbarrier.  The team's leader
+// (its thread 0) keeps a cursor over the rows the team will consume, issues
+// the first NSLOT copies up front and, each time the team has finished
+// reading a slot (after the team barrier of that row), refills it with the
+// row NSLOT places ahead.  Rows therefore stream through shared memory with no
+// registers held in flight and no producer warp (all 16 warps compute, and
+// each thread may use up to 128 registers).
 //
-// Thread t of a team owns B consecutive 16-element blocks of every row
-// (elements [16 B t, 16 B (t + 1))).  Its sum-of-squares partial is reduced by
-// a lane butterfly and then a pairwise tree over the team's warps, which
-// together form the balanced pairwise tree over the row's block partials (with
-// zero partials past the row end; adding +0 to a non-negative partial is
-// exact, so the padded tree equals the tree that carries an odd tail).
+// Thread t of a team owns the 32 consecutive elements [32 t, 32 t + 32) of
+// every row (two 16-element blocks).  Its sum-of-squares partial
+// b_{2t} + b_{2t+1} is reduced by a lane butterfly and then a pairwise tree
+// over the team's warps: together the balanced pairwise tree over the row's
+// block partials, with zero partials past the row end (adding +0 to a
+// non-negative partial is exact, so the padded tree equals the tree that
+// carries an odd tail up unchanged).
+//
+// Two copy paths fill a slot:
+//  - SWZ: H % 64 == 0.  The row is one 2-D tensor tile of 128-byte lines
+//    copied with SWIZZLE_128B, so the eight 16-byte chunks of each line land
+//    XOR-permuted by (line % 8); the consumer's 16-byte reads are then
+//    bank-conflict free with static register destinations.
+//  - plain: any H % 16 == 0.  1-D bulk copies; the consumer visits its four
+//    chunks in a lane-rotated order and undoes the rotation with selects.
 //
 // Every wait is bounded (2 s); a team whose wait runs out stops as a whole
-// (the abort flag travels with the reduction), the producer stops issuing,
-// drains the copies it has in flight and the kernel returns; the host sees
-// the flag through mb_device_status().
+// (the abort word is read after the team barrier), its leader drains the
+// copies it has in flight and the kernel returns; the host sees the flag
+// through mb_device_status().
 #pragma once
 
 #include "common.cuh"
 
 namespace mb {
 
-constexpr int kConsumerThreads = 512;     // per CTA, split into teams
-constexpr int kRingBytes = 196 * 1024;    // row slots per CTA (all teams)
+constexpr int kConsumerThreads = 512;     // per CTA (16 warps), split into teams
+constexpr int kRingBytes = 192 * 1024;    // row slots per CTA (all teams)
+constexpr int kSlotAlign = 1024;          // swizzle atom of SWIZZLE_128B
 
-// Shared-memory carve-up of one CTA (dynamic shared memory, 128-byte aligned
-// base).  Slots first (16-byte aligned for the bulk copies), then barriers,
-// then the reduction scratch.
+// The leader's copy cursor (kept in shared memory so that it costs the other
+// threads no registers): the next (token, slot) to examine, the next slot to
+// fill, and the counts of rows copied and consumed.
+struct RingCursor {
+    int ct, cj, wslot, issued, consumed, pad0, pad1, pad2;
+};
+
+// Shared-memory carve-up of one CTA.  The dynamic shared-memory base is
+// rounded up to kSlotAlign in the kernel (the launch asks for that much more).
 struct RingLayout {
     int nteam, nslot, slot_bytes, tw;
     __host__ __device__ size_t slots_bytes() const {
         return static_cast<size_t>(nteam) * nslot * slot_bytes;
     }
-    __host__ __device__ size_t bars_offset() const { return (slots_bytes() + 15) & ~size_t(15); }
+    __host__ __device__ size_t bars_offset() const { return slots_bytes(); }
     __host__ __device__ size_t red_offset() const {
-        return bars_offset() + static_cast<size_t>(nteam) * nslot * 2 * sizeof(uint64_t);
+        return bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t);
+    }
+    __host__ __device__ size_t abort_offset() const {
+        return red_offset() + static_cast<size_t>(nteam) * 2 * tw * sizeof(float);
+    }
+    __host__ __device__ size_t cursor_offset() const {
+        return abort_offset() + static_cast<size_t>(nteam) * 16;
     }
     __host__ __device__ size_t total_bytes() const {
-        // per team: [2][tw] float partials + [2][tw] int abort flags
-        return red_offset() + static_cast<size_t>(nteam) * 2 * tw * (sizeof(float) + sizeof(int));
+        return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;
     }
 };
+
+__host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
+
+// Row slot size: the row's BF16 bytes, rounded up to the swizzle atom.
+__host__ __device__ inline int slot_bytes_for(int H) { return round_up(2 * H, kSlotAlign); }
 
 // Team-wide sum of one float per thread, in the canonical tree order.  One
 // named barrier per call when the team spans several warps.
 template <int TW>
 struct TeamSum {
     float* red;        // [2][TW]
-    int* flags;        // [2][TW]
+    int* abort_word;   // one per team
     int bar_id;
     int warp_in_team;
     int lane;
@@ -62,69 +90,126 @@ struct TeamSum {
     // any thread passed fail = true.
     __device__ __forceinline__ float operator()(float v, bool fail, bool& abort) {
         v = warp_tree_sum(v);
-        const bool any_fail = __any_sync(0xffffffffu, fail);
         if constexpr (TW == 1) {
+            abort = __any_sync(0xffffffffu, fail);
             __syncwarp();
-            abort = any_fail;
             return v;
         } else {
-            if (lane == 0) {
-                red[buf * TW + warp_in_team] = v;
-                flags[buf * TW + warp_in_team] = any_fail ? 1 : 0;
-            }
+            if (fail) *reinterpret_cast<volatile int*>(abort_word) = 1;
+            if (lane == 0) red[buf * TW + warp_in_team] = v;
             named_bar_sync(bar_id, TW * 32);
             float p[TW];
-            int f = 0;
+            const float* src = red + buf * TW;
+            if constexpr (TW % 4 == 0) {
 #pragma unroll
-            for (int i = 0; i < TW; ++i) {
-                p[i] = red[buf * TW + i];
-                f |= flags[buf * TW + i];
+                for (int i = 0; i < TW; i += 4) {
+                    const float4 q = *reinterpret_cast<const float4*>(src + i);
+                    p[i] = q.x;
+                    p[i + 1] = q.y;
+                    p[i + 2] = q.z;
+                    p[i + 3] = q.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < TW; i += 2) {
+                    const float2 q = *reinterpret_cast<const float2*>(src + i);
+                    p[i] = q.x;
+                    p[i + 1] = q.y;
+                }
             }
+            abort = *reinterpret_cast<volatile int*>(abort_word) != 0;
             buf ^= 1;
-            abort = f != 0;
             return tree_sum_array<TW>(p);
         }
     }
 };
 
-// Reads this thread's B blocks (16 B * B bf16 values, 32 B per block) of a
-// row slot into 8 B 32-bit words (two BF16 each).  The 16-byte chunks are
-// visited in a lane-rotated order so that each quarter-warp touches all 32
-// banks once; the rotation is undone with selects (no dynamic register
-// indexing).
-template <int B>
-__device__ __forceinline__ void read_slot_blocks(const uint8_t* slot, int tid_in_team, int nvalid_blocks,
-                                                 uint32_t (&w)[8 * B]) {
-    constexpr int NCH = 2 * B;                      // 16-byte chunks per thread
-    const int shift = (B == 1) ? ((tid_in_team >> 2) & 1) : ((tid_in_team >> 1) & 3);
-    const uint8_t* base = slot + static_cast<size_t>(tid_in_team) * (32 * B);
-    uint4 r[NCH];
+// Reads this thread's 32 elements (16 words of two BF16) of a row slot.
+// nvalid (0..2) is the number of this thread's 16-element blocks inside the
+// row; chunks of missing blocks read as zero.
+template <bool SWZ>
+__device__ __forceinline__ void read_row32(uint32_t slot_saddr, int tid, int nvalid, uint32_t (&w)[16]) {
+    if constexpr (SWZ) {
+        const int line = tid >> 1;
+        const uint32_t base = slot_saddr + 128u * line;
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-        const int c = (i + shift) & (NCH - 1);
-        // chunk c belongs to block c / 2 of this thread
-        if (c / 2 < nvalid_blocks)
-            r[i] = *reinterpret_cast<const uint4*>(base + 16 * c);
-        else
-            r[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    // undo the rotation: chunk c was read at step (c - shift) mod NCH
+        for (int i = 0; i < 4; ++i) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (i / 2 < nvalid) {
+                const int cl = 4 * (tid & 1) + i;
+                v = lds128(base + 16u * static_cast<uint32_t>(cl ^ (line & 7)));
+            }
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+        }
+    } else {
+        const int shift = (tid >> 1) & 3;
+        const uint32_t base = slot_saddr + 64u * tid;
+        uint4 r[4];
 #pragma unroll
-    for (int bit = 1; bit < NCH; bit <<= 1) {
-        if (shift & bit) {
-            uint4 t[NCH];
+        for (int i = 0; i < 4; ++i) {
+            const int c = (i + shift) & 3;
+            r[i] = (c / 2 < nvalid) ? lds128(base + 16u * c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // chunk c was read at step (c - shift) mod 4
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) t[c] = r[(c + NCH - bit) & (NCH - 1)];
+        for (int bit = 1; bit < 4; bit <<= 1) {
+            if (shift & bit) {
+                uint4 t[4];
 #pragma unroll
-            for (int c = 0; c < NCH; ++c) r[c] = t[c];
+                for (int c = 0; c < 4; ++c) t[c] = r[(c + 4 - bit) & 3];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) r[c] = t[c];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            w[4 * c] = r[c].x;
+            w[4 * c + 1] = r[c].y;
+            w[4 * c + 2] = r[c].z;
+            w[4 * c + 3] = r[c].w;
         }
     }
+}
+
+// Sum-of-squares partial of this thread's two blocks: sequential fused
+// multiply-adds within each block (both chains advance together in one f32x2
+// operation), then b0 + b1.
+__device__ __forceinline__ float row32_sumsq(const uint32_t (&w)[16]) {
+    float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        w[4 * c + 0] = r[c].x;
-        w[4 * c + 1] = r[c].y;
-        w[4 * c + 2] = r[c].z;
-        w[4 * c + 3] = r[c].w;
+    for (int i = 0; i < 8; ++i) {
+        const float2 p = unpack_bf16x2(w[i]);       // block 0: elements 2i, 2i+1
+        const float2 q = unpack_bf16x2(w[8 + i]);   // block 1: elements 2i, 2i+1
+        const float2 lo = make_float2(p.x, q.x);
+        const float2 hi = make_float2(p.y, q.y);
+        a = fma2(lo, lo, a);
+        a = fma2(hi, hi, a);
+    }
+    return a.x + a.y;
+}
+
+// 1 / sqrt(ss / H + eps); when H is a power of two ss / H is the exact
+// product ss * (1 / H), which rounds like the division.
+__device__ __forceinline__ float inv_rms_h(float ss, float H, float rH, bool pow2, float eps) {
+    const float mean = pow2 ? __fmul_rn(ss, rH) : __fdiv_rn(ss, H);
+    return __frcp_rn(__fsqrt_rn(__fadd_rn(mean, eps)));
+}
+
+// Per-thread gain pairs g = center + w for this thread's 32 elements.
+__device__ __forceinline__ void load_gain32(const uint16_t* w, float center, int tid, int nvalid,
+                                            float2 (&g)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        if (w != nullptr && i / 8 < nvalid) {
+            const uint32_t word = *reinterpret_cast<const uint32_t*>(w + 32 * tid + 2 * i);
+            const float2 f = unpack_bf16x2(word);
+            g[i] = make_float2(__fadd_rn(center, f.x), __fadd_rn(center, f.y));
+        } else {
+            g[i] = make_float2(0.0f, 0.0f);
+        }
     }
 }
 

@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     const uint8_t* __restrict__ mask, int T, int E,
                                                     int k, int32_t* __restrict__ ids,
                                                     float* __restrict__ weights) {
+    griddep_wait();     // inputs may come from the previous kernel on the stream
+    griddep_launch();
     const int lane = threadIdx.x & 31;
     const int warp = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
@@ -165,13 +167,18 @@ cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* 
     int grid = (T + warps_per_cta - 1) / warps_per_cta;
     const int cap = device_info().sm_count * 8;
     if (grid > cap) grid = cap;
-    if (need <= 8)
-        route_kernel<8><<<grid, 256, 0, s>>>(logits, bias, mask, T, E, k, ids, weights);
-    else if (need <= 16)
-        route_kernel<16><<<grid, 256, 0, s>>>(logits, bias, mask, T, E, k, ids, weights);
-    else
-        route_kernel<32><<<grid, 256, 0, s>>>(logits, bias, mask, T, E, k, ids, weights);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (need <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8>, logits, bias, mask, T, E, k, ids, weights);
+    if (need <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16>, logits, bias, mask, T, E, k, ids, weights);
+    return cudaLaunchKernelEx(&cfg, route_kernel<32>, logits, bias, mask, T, E, k, ids, weights);
 }
 
 }  // namespace mb
