@@ -43,7 +43,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not is_stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, os.path.join(CSRC, "moe_boundary.cu"), "-o", tmp]
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.dirname(HEADER), os.path.join(CSRC, "moe_boundary.cu"),
+           "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

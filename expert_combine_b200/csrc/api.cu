@@ -4,7 +4,7 @@
 #include <cstdio>
 #include <mutex>
 
-#include "../../include/moe_boundary.h"
+#include "moe_boundary.h"
 #include "common.cuh"
 #include "internal.h"
 

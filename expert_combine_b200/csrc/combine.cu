@@ -128,7 +128,15 @@ __device__ __forceinline__ void join_token32(const uint32_t (&brw)[16], int t, i
     }
 }
 
-template <int TW, bool SWZ, bool JOIN>
+// One normalised BF16 pair: bf16((x * g) * inv).  With GC0 the gain is the
+// BF16 weight itself and x * w is formed exactly by a mixed-precision FMA.
+template <bool GC0>
+__device__ __forceinline__ uint32_t norm_word(uint32_t xw, uint32_t wpw, float2 gp, float2 inv2) {
+    const float2 t = GC0 ? mul_bf16x2_exact(xw, wpw) : mul2(unpack_bf16x2(xw), gp);
+    return pack_bf16x2_rn(mul2(t, inv2));
+}
+
+template <int TW, bool SWZ, bool JOIN, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     combine_kernel(const __grid_constant__ CUtensorMap tmap, const CombineArgs a) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
     const uint32_t ring_saddr = smem_addr(ring);
     uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
+    TeamSum<TW> team_sum{red_all + team * 4 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
 
     // ---- the leader's copy cursor over (token, slot): valid rows in order
     RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
@@ -200,11 +208,18 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         for (int i = 0; i < nslot; ++i) issue();
     }
 
+    // gain: with GC0 the packed BF16 weights, else FP32 pairs gc + w
+    uint32_t wp[16];
     float2 g[16];
-    load_gain32(a.w, a.gc, tid, nvalid, g);
+    if constexpr (GC0) {
+        load_words32(a.w + 32 * tid, nvalid > 0, nvalid > 1, wp);
+    } else {
+        load_gain32(a.w, a.gc, tid, nvalid, g);
+    }
     const float fH = static_cast<float>(H);
     const bool pow2 = (H & (H - 1)) == 0;
     const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
+    constexpr bool PAIR = GC0;   // two rows per team iteration (register budget allows it)
 
     // slot indices and weights of the token, one slot per lane (k <= 32),
     // loaded one token ahead
@@ -229,40 +244,80 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.0f, 0.0f);
 
-        for (int j = 0; j < k; ++j) {
-            const int32_t r = __shfl_sync(0xffffffffu, cur_r, j);
-            if (!slot_valid(r, R)) continue;
-            const float wj = __shfl_sync(0xffffffffu, cur_w, j);
-            const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
-            uint32_t wv[16];
+        // valid slots of this token, in slot order
+        unsigned vm = __ballot_sync(0xffffffffu, lane < k && slot_valid(cur_r, R));
+        while (vm != 0u) {
+            const int j0 = __ffs(vm) - 1;
+            vm &= vm - 1u;
+            const bool two = PAIR && vm != 0u;
+            int j1 = j0;
+            if (two) {
+                j1 = __ffs(vm) - 1;
+                vm &= vm - 1u;
+            }
+            const float w0 = __shfl_sync(0xffffffffu, cur_w, j0);
+            const float w1 = __shfl_sync(0xffffffffu, cur_w, j1);
+            int s1 = slot + 1, ph1 = phase;
+            if (s1 == nslot) {
+                s1 = 0;
+                ph1 ^= 1;
+            }
+            bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
+            if (two && ok) ok = mbar_wait_bounded(&tb[s1], ph1, 4u);
+            uint32_t wv0[16], wv1[16];
             if (ok) {
-                read_row32<SWZ>(ring_saddr + static_cast<uint32_t>(slot * slot_bytes), tid, nvalid, wv);
+                read_row32<SWZ>(ring_saddr + static_cast<uint32_t>(slot * slot_bytes), tid, nvalid, wv0);
+                if (two) read_row32<SWZ>(ring_saddr + static_cast<uint32_t>(s1 * slot_bytes), tid, nvalid, wv1);
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) wv[i] = 0u;
+                for (int i = 0; i < 16; ++i) wv0[i] = wv1[i] = 0u;
             }
             bool abort;
-            const float ss = team_sum(row32_sumsq(wv), !ok, abort);
+            float2 ss;
+            if (two) {
+                ss = team_sum.sum2(row32_sumsq(wv0), row32_sumsq(wv1), !ok, abort);
+            } else {
+                ss.x = team_sum(row32_sumsq(wv0), !ok, abort);
+                ss.y = ss.x;
+            }
             if (abort) {
                 aborted = true;
                 break;
             }
-            if (tid == 0) {   // the whole team has read this slot: refill it
-                cur->consumed += 1;
+            if (tid == 0) {   // the whole team has read these slots: refill them
+                cur->consumed += two ? 2 : 1;
                 fence_proxy_async_smem();
                 issue();
+                if (two) issue();
             }
-            if (++slot == nslot) {
-                slot = 0;
-                phase ^= 1;
+            slot = s1;
+            phase = ph1;
+            if (two) {
+                if (++slot == nslot) {
+                    slot = 0;
+                    phase ^= 1;
+                }
             }
-            const float inv = inv_rms_h(ss, fH, rH, pow2, a.eps);
-            const float2 inv2 = make_float2(inv, inv);
-            const float2 w2 = make_float2(wj, wj);
+            const float inv0 = inv_rms_h(ss.x, fH, rH, pow2, a.eps);
+            const float2 inv02 = make_float2(inv0, inv0);
+            const float2 w02 = make_float2(w0, w0);
+            if (two) {
+                const float inv1 = inv_rms_h(ss.y, fH, rH, pow2, a.eps);
+                const float2 inv12 = make_float2(inv1, inv1);
+                const float2 w12 = make_float2(w1, w1);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t y = pack_bf16x2_rn(mul2(mul2(unpack_bf16x2(wv[i]), g[i]), inv2));
-                acc[i] = fma2(w2, unpack_bf16x2(y), acc[i]);
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t y0 = norm_word<GC0>(wv0[i], wp[i], g[i], inv02);
+                    const uint32_t y1 = norm_word<GC0>(wv1[i], wp[i], g[i], inv12);
+                    acc[i] = fma2(w02, unpack_bf16x2(y0), acc[i]);
+                    acc[i] = fma2(w12, unpack_bf16x2(y1), acc[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t y0 = norm_word<GC0>(wv0[i], wp[i], g[i], inv02);
+                    acc[i] = fma2(w02, unpack_bf16x2(y0), acc[i]);
+                }
             }
         }
         if (aborted) break;
@@ -291,7 +346,7 @@ template <int TW>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     residual_join_kernel(const uint16_t* __restrict__ branch, int T, int H, JoinArgs join) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
-    __shared__ __align__(16) float red_all[NTEAM * 2 * TW];
+    __shared__ __align__(16) float red_all[NTEAM * 4 * TW];
     __shared__ int abort_all[NTEAM * 4];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -305,7 +360,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     __syncthreads();
     griddep_wait();
     griddep_launch();
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
+    TeamSum<TW> team_sum{red_all + team * 4 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
     const bool pow2 = (H & (H - 1)) == 0;
     const float rH = pow2 ? __frcp_rn(static_cast<float>(H)) : 0.0f;
     for (int t = blockIdx.x * NTEAM + team; t < T; t += gridDim.x * NTEAM) {
@@ -330,7 +385,7 @@ cudaLaunchConfig_t pdl_config(int grid, int block, size_t smem, cudaStream_t s, 
     return cfg;
 }
 
-template <int TW, bool SWZ, bool JOIN>
+template <int TW, bool SWZ, bool JOIN, bool GC0>
 cudaError_t launch_cb(const CUtensorMap& tmap, const CombineArgs& args, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
     const int slot_bytes = slot_bytes_for(args.H);
@@ -341,7 +396,7 @@ cudaError_t launch_cb(const CUtensorMap& tmap, const CombineArgs& args, cudaStre
     a.nslot = nslot;
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     const size_t smem = lay.total_bytes();
-    auto kern = combine_kernel<TW, SWZ, JOIN>;
+    auto kern = combine_kernel<TW, SWZ, JOIN, GC0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -353,16 +408,23 @@ cudaError_t launch_cb(const CUtensorMap& tmap, const CombineArgs& args, cudaStre
     return cudaLaunchKernelEx(&cfg, kern, tmap, a);
 }
 
-template <bool SWZ, bool JOIN>
+template <bool SWZ, bool JOIN, bool GC0>
 cudaError_t launch_cb_tw(int TW, const CUtensorMap& tmap, const CombineArgs& a, cudaStream_t s) {
     switch (TW) {
-        case 1: return launch_cb<1, SWZ, JOIN>(tmap, a, s);
-        case 2: return launch_cb<2, SWZ, JOIN>(tmap, a, s);
-        case 4: return launch_cb<4, SWZ, JOIN>(tmap, a, s);
-        case 8: return launch_cb<8, SWZ, JOIN>(tmap, a, s);
-        case 16: return launch_cb<16, SWZ, JOIN>(tmap, a, s);
+        case 1: return launch_cb<1, SWZ, JOIN, GC0>(tmap, a, s);
+        case 2: return launch_cb<2, SWZ, JOIN, GC0>(tmap, a, s);
+        case 4: return launch_cb<4, SWZ, JOIN, GC0>(tmap, a, s);
+        case 8: return launch_cb<8, SWZ, JOIN, GC0>(tmap, a, s);
+        case 16: return launch_cb<16, SWZ, JOIN, GC0>(tmap, a, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <bool SWZ, bool JOIN>
+cudaError_t launch_cb_gc(int TW, const CUtensorMap& tmap, const CombineArgs& a, cudaStream_t s) {
+    // gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
+    return a.gc == 0.0f ? launch_cb_tw<SWZ, JOIN, true>(TW, tmap, a, s)
+                        : launch_cb_tw<SWZ, JOIN, false>(TW, tmap, a, s);
 }
 
 template <int TW>
@@ -391,8 +453,8 @@ cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const i
                      encode_line_map(&tmap, expert_out, static_cast<uint64_t>(R) * (H / 64),
                                      static_cast<uint32_t>(H / 64));
     if (!swz) std::memset(&tmap, 0, sizeof(tmap));
-    if (swz) return fused ? launch_cb_tw<true, true>(TW, tmap, a, s) : launch_cb_tw<true, false>(TW, tmap, a, s);
-    return fused ? launch_cb_tw<false, true>(TW, tmap, a, s) : launch_cb_tw<false, false>(TW, tmap, a, s);
+    if (swz) return fused ? launch_cb_gc<true, true>(TW, tmap, a, s) : launch_cb_gc<true, false>(TW, tmap, a, s);
+    return fused ? launch_cb_gc<false, true>(TW, tmap, a, s) : launch_cb_gc<false, false>(TW, tmap, a, s);
 }
 
 cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,

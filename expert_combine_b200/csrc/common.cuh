@@ -238,6 +238,31 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
     return bits_f2(d);
 }
+// Mixed-precision fused multiply-add on the BF16 halves of two pair words:
+// fl32(a_h * b_h + c), the product exact (BF16 inputs widen exactly), one
+// rounding -- the same bits as fmaf(float(a_h), float(b_h), c).
+__device__ __forceinline__ float fma_bf16_lo(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+// Exact product of the BF16 halves as a float pair: (a_lo * b_lo, a_hi * b_hi)
+// (adding -0 keeps the sign of a zero product).
+__device__ __forceinline__ float2 mul_bf16x2_exact(uint32_t a, uint32_t b) {
+    return make_float2(fma_bf16_lo(a, b, -0.0f), fma_bf16_hi(a, b, -0.0f));
+}
+
 // BF16 pair word -> two floats (exact).
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));

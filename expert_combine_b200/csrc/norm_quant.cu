@@ -29,7 +29,7 @@ struct NormQuantArgs {
     int nslot;
 };
 
-template <int TW, bool SWZ>
+template <int TW, bool SWZ, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     norm_quant_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
     const uint32_t ring_saddr = smem_addr(ring);
     uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
-    TeamSum<TW> team_sum{red_all + team * 2 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
+    TeamSum<TW> team_sum{red_all + team * 4 * TW, abort_all + 4 * team, 1 + team, warp_in_team, lane, 0};
 
     // ---- the leader's copy cursor: one row (tp segments) per token
     const int hs = H / a.tp;
@@ -96,8 +96,23 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         for (int i = 0; i < nslot; ++i) issue();
     }
 
+    // gain: with GC0 the packed BF16 weights (x * w formed exactly by a
+    // mixed-precision FMA), else FP32 pairs gc + w
+    uint32_t wp[16];
     float2 g[16];
-    load_gain32(a.w, a.gc, tid, nvalid, g);
+    if constexpr (GC0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (c / 2 < nvalid) v = *reinterpret_cast<const uint4*>(a.w + 32 * tid + 8 * c);
+            wp[4 * c] = v.x;
+            wp[4 * c + 1] = v.y;
+            wp[4 * c + 2] = v.z;
+            wp[4 * c + 3] = v.w;
+        }
+    } else {
+        load_gain32(a.w, a.gc, tid, nvalid, g);
+    }
     const float gs = __ldg(a.gs);
     const float rgs = __frcp_rn(gs);
     constexpr float kR6 = (float)(1.0 / 6.0);
@@ -138,7 +153,9 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 uint32_t m = 0u;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float2 t2 = mul2(mul2(unpack_bf16x2(wv[8 * b + i]), g[8 * b + i]), inv2);
+                    const float2 xg = GC0 ? mul_bf16x2_exact(wv[8 * b + i], wp[8 * b + i])
+                                          : mul2(unpack_bf16x2(wv[8 * b + i]), g[8 * b + i]);
+                    const float2 t2 = mul2(xg, inv2);
                     yw[i] = pack_bf16x2_rn(t2);
                     m = maxabs_bf16x2(m, yw[i]);
                 }
@@ -173,7 +190,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 
 namespace {
 
-template <int TW, bool SWZ>
+template <int TW, bool SWZ, bool GC0>
 cudaError_t launch_nq(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
     const int slot_bytes = slot_bytes_for(args.H);
@@ -184,7 +201,7 @@ cudaError_t launch_nq(const CUtensorMap& tmap, const NormQuantArgs& args, cudaSt
     a.nslot = nslot;
     const RingLayout lay{NTEAM, nslot, slot_bytes, TW};
     const size_t smem = lay.total_bytes();
-    auto kern = norm_quant_kernel<TW, SWZ>;
+    auto kern = norm_quant_kernel<TW, SWZ, GC0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -204,16 +221,22 @@ cudaError_t launch_nq(const CUtensorMap& tmap, const NormQuantArgs& args, cudaSt
     return cudaLaunchKernelEx(&cfg, kern, tmap, a);
 }
 
-template <bool SWZ>
+template <bool SWZ, bool GC0>
 cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
     switch (TW) {
-        case 1: return launch_nq<1, SWZ>(tmap, a, s);
-        case 2: return launch_nq<2, SWZ>(tmap, a, s);
-        case 4: return launch_nq<4, SWZ>(tmap, a, s);
-        case 8: return launch_nq<8, SWZ>(tmap, a, s);
-        case 16: return launch_nq<16, SWZ>(tmap, a, s);
+        case 1: return launch_nq<1, SWZ, GC0>(tmap, a, s);
+        case 2: return launch_nq<2, SWZ, GC0>(tmap, a, s);
+        case 4: return launch_nq<4, SWZ, GC0>(tmap, a, s);
+        case 8: return launch_nq<8, SWZ, GC0>(tmap, a, s);
+        case 16: return launch_nq<16, SWZ, GC0>(tmap, a, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
+template <bool SWZ>
+cudaError_t launch_nq_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
+    return a.gc == 0.0f ? launch_nq_tw<SWZ, true>(TW, tmap, a, s) : launch_nq_tw<SWZ, false>(TW, tmap, a, s);
 }
 
 }  // namespace
@@ -239,9 +262,9 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
     CUtensorMap tmap;
     if (swz && encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64),
                                static_cast<uint32_t>(hs / 64)))
-        return launch_nq_tw<true>(team_warps(H), tmap, a, s);
+        return launch_nq_gc<true>(team_warps(H), tmap, a, s);
     std::memset(&tmap, 0, sizeof(tmap));
-    return launch_nq_tw<false>(team_warps(H), tmap, a, s);
+    return launch_nq_gc<false>(team_warps(H), tmap, a, s);
 }
 
 }  // namespace mb

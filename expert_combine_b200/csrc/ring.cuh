@@ -57,10 +57,10 @@ struct RingLayout {
     }
     __host__ __device__ size_t bars_offset() const { return slots_bytes(); }
     __host__ __device__ size_t red_offset() const {
-        return bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t);
+        return (bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t) + 15) & ~size_t(15);
     }
     __host__ __device__ size_t abort_offset() const {
-        return red_offset() + static_cast<size_t>(nteam) * 2 * tw * sizeof(float);
+        return red_offset() + static_cast<size_t>(nteam) * 2 * tw * sizeof(float2);
     }
     __host__ __device__ size_t cursor_offset() const {
         return abort_offset() + static_cast<size_t>(nteam) * 16;
@@ -79,7 +79,7 @@ __host__ __device__ inline int slot_bytes_for(int H) { return round_up(2 * H, kS
 // named barrier per call when the team spans several warps.
 template <int TW>
 struct TeamSum {
-    float* red;        // [2][TW]
+    float* red;        // [2][TW] float2 (two partials per warp)
     int* abort_word;   // one per team
     int bar_id;
     int warp_in_team;
@@ -96,30 +96,52 @@ struct TeamSum {
             return v;
         } else {
             if (fail) *reinterpret_cast<volatile int*>(abort_word) = 1;
-            if (lane == 0) red[buf * TW + warp_in_team] = v;
+            if (lane == 0) red[buf * 2 * TW + warp_in_team] = v;
             named_bar_sync(bar_id, TW * 32);
             float p[TW];
-            const float* src = red + buf * TW;
-            if constexpr (TW % 4 == 0) {
+            const float* src = red + buf * 2 * TW;
 #pragma unroll
-                for (int i = 0; i < TW; i += 4) {
-                    const float4 q = *reinterpret_cast<const float4*>(src + i);
-                    p[i] = q.x;
-                    p[i + 1] = q.y;
-                    p[i + 2] = q.z;
-                    p[i + 3] = q.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < TW; i += 2) {
-                    const float2 q = *reinterpret_cast<const float2*>(src + i);
-                    p[i] = q.x;
-                    p[i + 1] = q.y;
-                }
+            for (int i = 0; i < TW; i += 2) {
+                const float2 q = *reinterpret_cast<const float2*>(src + i);
+                p[i] = q.x;
+                p[i + 1] = q.y;
             }
             abort = *reinterpret_cast<volatile int*>(abort_word) != 0;
             buf ^= 1;
             return tree_sum_array<TW>(p);
+        }
+    }
+
+    // Two independent sums with one barrier.
+    __device__ __forceinline__ float2 sum2(float v0, float v1, bool fail, bool& abort) {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o0 = __shfl_xor_sync(0xffffffffu, v0, off);
+            const float o1 = __shfl_xor_sync(0xffffffffu, v1, off);
+            v0 = v0 + o0;
+            v1 = v1 + o1;
+        }
+        if constexpr (TW == 1) {
+            abort = __any_sync(0xffffffffu, fail);
+            __syncwarp();
+            return make_float2(v0, v1);
+        } else {
+            if (fail) *reinterpret_cast<volatile int*>(abort_word) = 1;
+            float2* src2 = reinterpret_cast<float2*>(red) + buf * TW;
+            if (lane == 0) src2[warp_in_team] = make_float2(v0, v1);
+            named_bar_sync(bar_id, TW * 32);
+            float p0[TW], p1[TW];
+#pragma unroll
+            for (int i = 0; i < TW; i += 2) {
+                const float4 q = *reinterpret_cast<const float4*>(src2 + i);
+                p0[i] = q.x;
+                p1[i] = q.y;
+                p0[i + 1] = q.z;
+                p1[i + 1] = q.w;
+            }
+            abort = *reinterpret_cast<volatile int*>(abort_word) != 0;
+            buf ^= 1;
+            return make_float2(tree_sum_array<TW>(p0), tree_sum_array<TW>(p1));
         }
     }
 };
@@ -175,20 +197,18 @@ __device__ __forceinline__ void read_row32(uint32_t slot_saddr, int tid, int nva
 }
 
 // Sum-of-squares partial of this thread's two blocks: sequential fused
-// multiply-adds within each block (both chains advance together in one f32x2
-// operation), then b0 + b1.
+// multiply-adds within each block (BF16 inputs, FP32 accumulator), then
+// b0 + b1.
 __device__ __forceinline__ float row32_sumsq(const uint32_t (&w)[16]) {
-    float2 a = make_float2(0.0f, 0.0f);
+    float b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float2 p = unpack_bf16x2(w[i]);       // block 0: elements 2i, 2i+1
-        const float2 q = unpack_bf16x2(w[8 + i]);   // block 1: elements 2i, 2i+1
-        const float2 lo = make_float2(p.x, q.x);
-        const float2 hi = make_float2(p.y, q.y);
-        a = fma2(lo, lo, a);
-        a = fma2(hi, hi, a);
+        b0 = fma_bf16_lo(w[i], w[i], b0);           // block 0: element 2i
+        b1 = fma_bf16_lo(w[8 + i], w[8 + i], b1);   // block 1: element 2i
+        b0 = fma_bf16_hi(w[i], w[i], b0);           // element 2i + 1
+        b1 = fma_bf16_hi(w[8 + i], w[8 + i], b1);
     }
-    return a.x + a.y;
+    return b0 + b1;
 }
 
 // 1 / sqrt(ss / H + eps); when H is a power of two ss / H is the exact
