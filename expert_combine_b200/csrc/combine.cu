@@ -128,12 +128,13 @@ __device__ __forceinline__ void join_token32(const uint32_t (&brw)[16], int t, i
     }
 }
 
-// One normalised BF16 pair: bf16((x * g) * inv).  With GC0 the gain is the
-// BF16 weight itself and x * w is formed exactly by a mixed-precision FMA.
+// One normalised pair as BF16-exact floats: bf16((x * g) * inv).  With GC0
+// the gain is the BF16 weight itself and x * w is formed exactly by a
+// mixed-precision FMA.
 template <bool GC0>
-__device__ __forceinline__ uint32_t norm_word(uint32_t xw, uint32_t wpw, float2 gp, float2 inv2) {
+__device__ __forceinline__ float2 norm_pair(uint32_t xw, uint32_t wpw, float2 gp, float2 inv2) {
     const float2 t = GC0 ? mul_bf16x2_exact(xw, wpw) : mul2(unpack_bf16x2(xw), gp);
-    return pack_bf16x2_rn(mul2(t, inv2));
+    return round_bf16_f2(mul2(t, inv2));
 }
 
 template <int TW, bool SWZ, bool JOIN, bool GC0>
@@ -307,16 +308,15 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 const float2 w12 = make_float2(w1, w1);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint32_t y0 = norm_word<GC0>(wv0[i], wp[i], g[i], inv02);
-                    const uint32_t y1 = norm_word<GC0>(wv1[i], wp[i], g[i], inv12);
-                    acc[i] = fma2(w02, unpack_bf16x2(y0), acc[i]);
-                    acc[i] = fma2(w12, unpack_bf16x2(y1), acc[i]);
+                    const float2 y0 = norm_pair<GC0>(wv0[i], wp[i], g[i], inv02);
+                    const float2 y1 = norm_pair<GC0>(wv1[i], wp[i], g[i], inv12);
+                    acc[i] = fma2(w02, y0, acc[i]);
+                    acc[i] = fma2(w12, y1, acc[i]);
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint32_t y0 = norm_word<GC0>(wv0[i], wp[i], g[i], inv02);
-                    acc[i] = fma2(w02, unpack_bf16x2(y0), acc[i]);
+                    acc[i] = fma2(w02, norm_pair<GC0>(wv0[i], wp[i], g[i], inv02), acc[i]);
                 }
             }
         }
@@ -336,6 +336,224 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         if constexpr (JOIN) join_token32<TW>(brw, t, H, tid, nvalid, a.join, team_sum, pow2, rH);
     }
     // copies still in flight (only after an abort) land before the CTA exits
+    if (tid == 0)
+        for (int f = cur->consumed; f < cur->issued; ++f)
+            mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+}
+
+// ---------------------------------------------------------------------------
+// Wide-row combine (H >= 2048, H % 64 == 0): thread t of a team owns the
+// 128-byte line t of every row (64 elements, four 16-element blocks), so a
+// team of P = H/64 (rounded up to a power of two) threads covers a row and a
+// CTA holds 512/P teams.  Each row is read twice from its shared-memory slot:
+// pass 1 forms the sum-of-squares partial (the team barrier then yields inv),
+// pass 2 re-reads the row, normalises it and accumulates; only the FP32
+// accumulator lives in registers.  A slot is handed back one row late (at the
+// barrier of the team's next row, when every warp has finished pass 2), and
+// the packed BF16 weights sit in a shared-memory table laid out so that both
+// the swizzled row lines and the table are read without bank conflicts.
+struct WideLayout {
+    int nteam, nslot, slot_bytes, P;
+    __host__ __device__ size_t slots_bytes() const { return static_cast<size_t>(nteam) * nslot * slot_bytes; }
+    __host__ __device__ size_t wtab_offset() const { return slots_bytes(); }              // [8][P] x 16 B
+    __host__ __device__ size_t bars_offset() const { return wtab_offset() + static_cast<size_t>(P) * 128; }
+    __host__ __device__ size_t part_offset() const {                                      // [nteam][2][TW] f32
+        return (bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t) + 15) & ~size_t(15);
+    }
+    __host__ __device__ size_t abort_offset() const { return part_offset() + static_cast<size_t>(nteam) * 2 * (P / 32) * sizeof(float); }
+    __host__ __device__ size_t cursor_offset() const { return abort_offset() + static_cast<size_t>(nteam) * 16; }
+    __host__ __device__ size_t total_bytes() const {
+        return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;
+    }
+};
+
+template <int TW, bool GC0>
+__global__ void __launch_bounds__(kConsumerThreads, 1)
+    combine_wide_kernel(const __grid_constant__ CUtensorMap tmap, const CombineArgs a) {
+    constexpr int P = TW * 32;
+    constexpr int NTEAM = kConsumerThreads / P;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_saddr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_saddr + kSlotAlign - 1) & ~uint32_t(kSlotAlign - 1)) - raw_saddr);
+    const int H = a.H;
+    const int nslot = a.nslot;
+    const int slot_bytes = slot_bytes_for(H);
+    const WideLayout lay{NTEAM, nslot, slot_bytes, P};
+    uint4* wtab = reinterpret_cast<uint4*>(smem + lay.wtab_offset());
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
+    float* part_all = reinterpret_cast<float*>(smem + lay.part_offset());
+    int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int team = warp / TW;
+    const int warp_in_team = warp % TW;
+    const int tid = warp_in_team * 32 + lane;
+    const int lines = H / 64;
+    const bool has_line = tid < lines;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    griddep_wait();     // row indices and weights may come from the previous kernel
+    griddep_launch();
+    if (team == 0) {    // the weight table, chunk c of line t at [c][t]
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            wtab[c * P + tid] = has_line ? *reinterpret_cast<const uint4*>(a.w + 64 * tid + 8 * c)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+
+    const int T = a.T, k = a.k;
+    const int64_t R = a.R;
+    const int team_stride = gridDim.x * NTEAM;
+    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
+    const uint32_t ring_saddr = smem_addr(ring);
+    const uint32_t wtab_saddr = smem_addr(wtab);
+    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
+    int* abort_word = abort_all + 4 * team;
+    float* part = part_all + team * 2 * TW;
+
+    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
+    auto issue = [&]() {
+        int ct = cur->ct, cj = cur->cj;
+        while (ct < T) {
+            const int32_t r = __ldg(a.row_idx + static_cast<size_t>(ct) * k + cj);
+            if (++cj == k) {
+                cj = 0;
+                ct += team_stride;
+                if (ct + team_stride < T)
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.row_idx + static_cast<size_t>(ct + team_stride) * k));
+            }
+            if (!slot_valid(r, R)) continue;
+            const int ws = cur->wslot;
+            mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
+            tma_load_2d(smem_addr(ring + static_cast<size_t>(ws) * slot_bytes), &tmap, 0, r * lines, &tb[ws]);
+            cur->issued += 1;
+            cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
+            break;
+        }
+        cur->ct = ct;
+        cur->cj = cj;
+    };
+    if (tid == 0) {
+        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < nslot; ++i) issue();
+    }
+
+    const float fH = static_cast<float>(H);
+    const bool pow2 = (H & (H - 1)) == 0;
+    const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
+    const float2 gc2 = make_float2(a.gc, a.gc);
+    // swizzled position of chunk c of this thread's line (SWIZZLE_128B)
+    const uint32_t line_off = 128u * static_cast<uint32_t>(tid);
+    const int sw = tid & 7;
+
+    int t = blockIdx.x * NTEAM + team;
+    int32_t my_r = -1;
+    float my_w = 0.0f;
+    if (t < T && lane < k) {
+        my_r = __ldg(a.row_idx + static_cast<size_t>(t) * k + lane);
+        my_w = __ldg(a.wt + static_cast<size_t>(t) * k + lane);
+    }
+    int slot = 0, phase = 0, pbuf = 0;
+    bool held = false;      // a slot waits to be handed back at the next barrier
+    bool aborted = false;
+    float2 acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+
+    for (; t < T; t += team_stride) {
+        const int32_t cur_r = my_r;
+        const float cur_w = my_w;
+        const int tn = t + team_stride;
+        if (tn < T && lane < k) {
+            my_r = __ldg(a.row_idx + static_cast<size_t>(tn) * k + lane);
+            my_w = __ldg(a.wt + static_cast<size_t>(tn) * k + lane);
+        }
+        unsigned vm = __ballot_sync(0xffffffffu, lane < k && slot_valid(cur_r, R));
+        while (vm != 0u) {
+            const int j = __ffs(vm) - 1;
+            vm &= vm - 1u;
+            const float wj = __shfl_sync(0xffffffffu, cur_w, j);
+            const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
+            const uint32_t sbase = ring_saddr + static_cast<uint32_t>(slot * slot_bytes) + line_off;
+            // pass 1: sum of squares of the four blocks, two chunks per block
+            float b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (ok && has_line) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = lds128(sbase + 16u * static_cast<uint32_t>(c ^ sw));
+                    float& acc_b = b[c >> 1];
+                    acc_b = fma_bf16_lo(v.x, v.x, acc_b);
+                    acc_b = fma_bf16_hi(v.x, v.x, acc_b);
+                    acc_b = fma_bf16_lo(v.y, v.y, acc_b);
+                    acc_b = fma_bf16_hi(v.y, v.y, acc_b);
+                    acc_b = fma_bf16_lo(v.z, v.z, acc_b);
+                    acc_b = fma_bf16_hi(v.z, v.z, acc_b);
+                    acc_b = fma_bf16_lo(v.w, v.w, acc_b);
+                    acc_b = fma_bf16_hi(v.w, v.w, acc_b);
+                }
+            }
+            if (!ok) *reinterpret_cast<volatile int*>(abort_word) = 1;
+            const float v = warp_tree_sum((b[0] + b[1]) + (b[2] + b[3]));
+            if (lane == 0) part[pbuf * TW + warp_in_team] = v;
+            if constexpr (TW == 1) __syncwarp();
+            else named_bar_sync(1 + team, P);
+            if (*reinterpret_cast<volatile int*>(abort_word) != 0) {
+                aborted = true;
+                break;
+            }
+            if (tid == 0 && held) {   // every warp has finished pass 2 of the previous row
+                cur->consumed += 1;
+                fence_proxy_async_smem();
+                issue();
+            }
+            held = true;
+            float pp[TW];
+#pragma unroll
+            for (int i = 0; i < TW; ++i) pp[i] = part[pbuf * TW + i];
+            pbuf ^= 1;
+            const float inv = inv_rms_h(tree_sum_array<TW>(pp), fH, rH, pow2, a.eps);
+            const float2 inv2 = make_float2(inv, inv);
+            const float2 w2 = make_float2(wj, wj);
+            // pass 2: normalise and accumulate
+            if (has_line) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 x = lds128(sbase + 16u * static_cast<uint32_t>(c ^ sw));
+                    const uint4 wv = lds128(wtab_saddr + 16u * static_cast<uint32_t>(c * P + tid));
+                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+                    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 xg = GC0 ? mul_bf16x2_exact(xs[q], ws[q])
+                                              : mul2(unpack_bf16x2(xs[q]), add2(gc2, unpack_bf16x2(ws[q])));
+                        acc[4 * c + q] = fma2(w2, round_bf16_f2(mul2(xg, inv2)), acc[4 * c + q]);
+                    }
+                }
+            }
+            if (++slot == nslot) {
+                slot = 0;
+                phase ^= 1;
+            }
+        }
+        if (aborted) break;
+        if (has_line && a.out != nullptr) {
+            uint16_t* orow = a.out + static_cast<size_t>(t) * H + 64 * tid;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(orow + 8 * c) =
+                    make_uint4(pack_bf16x2_rn(acc[4 * c]), pack_bf16x2_rn(acc[4 * c + 1]),
+                               pack_bf16x2_rn(acc[4 * c + 2]), pack_bf16x2_rn(acc[4 * c + 3]));
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
+    }
+    // copies still in flight land before the CTA exits
     if (tid == 0)
         for (int f = cur->consumed; f < cur->issued; ++f)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
@@ -427,6 +645,44 @@ cudaError_t launch_cb_gc(int TW, const CUtensorMap& tmap, const CombineArgs& a, 
                         : launch_cb_tw<SWZ, JOIN, false>(TW, tmap, a, s);
 }
 
+template <int TW, bool GC0>
+cudaError_t launch_wide(const CUtensorMap& tmap, const CombineArgs& args, cudaStream_t s) {
+    constexpr int P = TW * 32;
+    constexpr int NTEAM = kConsumerThreads / P;
+    const int slot_bytes = slot_bytes_for(args.H);
+    WideLayout lay{NTEAM, 1, slot_bytes, P};
+    const size_t fixed = lay.total_bytes() - static_cast<size_t>(NTEAM) * slot_bytes;
+    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - 64 * NTEAM;
+    int nslot = avail / (NTEAM * slot_bytes);
+    if (nslot > 16) nslot = 16;
+    if (nslot < 2) return cudaErrorInvalidConfiguration;
+    lay.nslot = nslot;
+    CombineArgs a = args;
+    a.nslot = nslot;
+    const size_t smem = lay.total_bytes();
+    auto kern = combine_wide_kernel<TW, GC0>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int grid = (a.T + NTEAM - 1) / NTEAM;
+    const int cap = device_info().sm_count;
+    if (grid > cap) grid = cap;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pdl_config(grid, kConsumerThreads, smem, s, attr);
+    return cudaLaunchKernelEx(&cfg, kern, tmap, a);
+}
+
+template <bool GC0>
+cudaError_t launch_wide_tw(int TW, const CUtensorMap& tmap, const CombineArgs& a, cudaStream_t s) {
+    switch (TW) {
+        case 1: return launch_wide<1, GC0>(tmap, a, s);
+        case 2: return launch_wide<2, GC0>(tmap, a, s);
+        case 4: return launch_wide<4, GC0>(tmap, a, s);
+        case 8: return launch_wide<8, GC0>(tmap, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int TW>
 cudaError_t launch_rj(const uint16_t* branch, int T, int H, const JoinArgs& join, cudaStream_t s) {
     constexpr int NTEAM = kConsumerThreads / (TW * 32);
@@ -453,6 +709,12 @@ cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const i
                      encode_line_map(&tmap, expert_out, static_cast<uint64_t>(R) * (H / 64),
                                      static_cast<uint32_t>(H / 64));
     if (!swz) std::memset(&tmap, 0, sizeof(tmap));
+    if (swz && !fused && H >= 2048) {
+        // one 128-byte line per thread: P = next_pow2(H / 64) threads per team
+        int P = 32;
+        while (P < H / 64) P <<= 1;
+        return a.gc == 0.0f ? launch_wide_tw<true>(P / 32, tmap, a, s) : launch_wide_tw<false>(P / 32, tmap, a, s);
+    }
     if (swz) return fused ? launch_cb_gc<true, true>(TW, tmap, a, s) : launch_cb_gc<true, false>(TW, tmap, a, s);
     return fused ? launch_cb_gc<false, true>(TW, tmap, a, s) : launch_cb_gc<false, false>(TW, tmap, a, s);
 }

@@ -273,6 +273,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float2 v) {
     asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(v.x), "f"(v.y));
     return r;
 }
+// Round one float to BF16 (nearest even) and return it as a float: the
+// conversion packs (a, 0) so the result word is exactly the float's bits.
+__device__ __forceinline__ float round_bf16_f(float a) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(0.0f));
+    return __uint_as_float(r);
+}
+__device__ __forceinline__ float2 round_bf16_f2(float2 v) {
+    return make_float2(round_bf16_f(v.x), round_bf16_f(v.y));
+}
+
 // Largest magnitude of the two BF16 halves of a and b, per half (signs are
 // not meaningful in the result; only the magnitudes are used).
 __device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {

@@ -62,8 +62,11 @@ struct RingLayout {
     __host__ __device__ size_t abort_offset() const {
         return red_offset() + static_cast<size_t>(nteam) * 2 * tw * sizeof(float2);
     }
-    __host__ __device__ size_t cursor_offset() const {
+    __host__ __device__ size_t pipe_offset() const {   // [nteam][2][tw] row partials
         return abort_offset() + static_cast<size_t>(nteam) * 16;
+    }
+    __host__ __device__ size_t cursor_offset() const {
+        return pipe_offset() + static_cast<size_t>(nteam) * 2 * tw * sizeof(float);
     }
     __host__ __device__ size_t total_bytes() const {
         return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;

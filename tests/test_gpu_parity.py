@@ -82,6 +82,16 @@ def test_combine_shapes(cuda_dev, H, k):
     check_combine(case)
 
 
+@pytest.mark.parametrize("H", [1024, 2688, 8192])
+def test_combine_gain_centre_one(cuda_dev, H):
+    case = synth.make_case("tiny", device=cuda_dev, T=29, H=H, join=False)
+    g = torch.Generator(device=cuda_dev)
+    g.manual_seed(7)
+    case.post_w.copy_((0.1 * torch.randn(H, generator=g, device=cuda_dev)).to(torch.bfloat16))
+    case.post_gc = 1.0
+    check_combine(case)
+
+
 def test_combine_invalid_slots_never_read(cuda_dev):
     case = synth.make_case("tiny", device=cuda_dev)
     idx = case.row_idx
