@@ -352,21 +352,6 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // barrier of the team's next row, when every warp has finished pass 2), and
 // the packed BF16 weights sit in a shared-memory table laid out so that both
 // the swizzled row lines and the table are read without bank conflicts.
-struct WideLayout {
-    int nteam, nslot, slot_bytes, P;
-    __host__ __device__ size_t slots_bytes() const { return static_cast<size_t>(nteam) * nslot * slot_bytes; }
-    __host__ __device__ size_t wtab_offset() const { return slots_bytes(); }              // [8][P] x 16 B
-    __host__ __device__ size_t bars_offset() const { return wtab_offset() + static_cast<size_t>(P) * 128; }
-    __host__ __device__ size_t part_offset() const {                                      // [nteam][2][TW] f32
-        return (bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t) + 15) & ~size_t(15);
-    }
-    __host__ __device__ size_t abort_offset() const { return part_offset() + static_cast<size_t>(nteam) * 2 * (P / 32) * sizeof(float); }
-    __host__ __device__ size_t cursor_offset() const { return abort_offset() + static_cast<size_t>(nteam) * 16; }
-    __host__ __device__ size_t total_bytes() const {
-        return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;
-    }
-};
-
 template <int TW, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     combine_wide_kernel(const __grid_constant__ CUtensorMap tmap, const CombineArgs a) {

@@ -188,6 +188,186 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
 }
 
+// ---------------------------------------------------------------------------
+// Wide-row norm-quant (H >= 2048, H % 64 == 0, tensor-map copies): thread t of
+// a team owns the 128-byte line t of every row (four 16-element blocks) and
+// keeps its 32 words in registers across the team barrier, so the slot is
+// refilled as soon as the barrier has passed.  The packed BF16 weights sit in
+// a shared-memory table read without bank conflicts.
+template <int TW, bool GC0>
+__global__ void __launch_bounds__(kConsumerThreads, 1)
+    norm_quant_wide_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
+    constexpr int P = TW * 32;
+    constexpr int NTEAM = kConsumerThreads / P;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_saddr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_saddr + kSlotAlign - 1) & ~uint32_t(kSlotAlign - 1)) - raw_saddr);
+    const int H = a.H;
+    const int nslot = a.nslot;
+    const int slot_bytes = slot_bytes_for(H);
+    const WideLayout lay{NTEAM, nslot, slot_bytes, P};
+    uint4* wtab = reinterpret_cast<uint4*>(smem + lay.wtab_offset());
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
+    float* part_all = reinterpret_cast<float*>(smem + lay.part_offset());
+    int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int team = warp / TW;
+    const int warp_in_team = warp % TW;
+    const int tid = warp_in_team * 32 + lane;
+    const int lines = H / 64;
+    const bool has_line = tid < lines;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    griddep_wait();     // inputs may come from the previous kernel on the stream
+    griddep_launch();
+    if (team == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            wtab[c * P + tid] = has_line ? *reinterpret_cast<const uint4*>(a.w + 64 * tid + 8 * c)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+
+    const int M = a.M;
+    const int team_stride = gridDim.x * NTEAM;
+    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
+    const uint32_t ring_saddr = smem_addr(ring);
+    const uint32_t wtab_saddr = smem_addr(wtab);
+    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
+    int* abort_word = abort_all + 4 * team;
+    float* part = part_all + team * 2 * TW;
+
+    // ---- the leader's copy cursor: one row (tp segments) per token
+    const int hs = H / a.tp;
+    const int seg_lines = hs / 64;
+    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
+    auto issue = [&]() {
+        const int nt = cur->ct;
+        if (nt >= M) return;
+        const int ws = cur->wslot;
+        mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
+        uint8_t* dst = ring + static_cast<size_t>(ws) * slot_bytes;
+        for (int s = 0; s < a.tp; ++s)
+            tma_load_2d(smem_addr(dst + static_cast<size_t>(s) * 2 * hs), &tmap, 0, (s * M + nt) * seg_lines,
+                        &tb[ws]);
+        cur->ct = nt + team_stride;
+        cur->issued += 1;
+        cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
+    };
+    if (tid == 0) {
+        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < nslot; ++i) issue();
+    }
+
+    const float gs = __ldg(a.gs);
+    const float rgs = __frcp_rn(gs);
+    constexpr float kR6 = (float)(1.0 / 6.0);
+    const float fH = static_cast<float>(H);
+    const bool pow2 = (H & (H - 1)) == 0;
+    const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
+    const float2 zero2 = make_float2(0.0f, 0.0f);
+    const float2 gc2 = make_float2(a.gc, a.gc);
+    const uint32_t line_off = 128u * static_cast<uint32_t>(tid);
+    const int sw = tid & 7;
+    const int nblocks = H / 16;
+
+    int slot = 0, phase = 0, pbuf = 0;
+    for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride) {
+        const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
+        uint32_t wv[32];
+        float b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint32_t sbase = ring_saddr + static_cast<uint32_t>(slot * slot_bytes) + line_off;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (ok && has_line) v = lds128(sbase + 16u * static_cast<uint32_t>(c ^ sw));
+            wv[4 * c] = v.x;
+            wv[4 * c + 1] = v.y;
+            wv[4 * c + 2] = v.z;
+            wv[4 * c + 3] = v.w;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            float& acc_b = b[c >> 1];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc_b = fma_bf16_lo(wv[4 * c + q], wv[4 * c + q], acc_b);
+                acc_b = fma_bf16_hi(wv[4 * c + q], wv[4 * c + q], acc_b);
+            }
+        }
+        if (!ok) *reinterpret_cast<volatile int*>(abort_word) = 1;
+        const float v = warp_tree_sum((b[0] + b[1]) + (b[2] + b[3]));
+        if (lane == 0) part[pbuf * TW + warp_in_team] = v;
+        if constexpr (TW == 1) __syncwarp();
+        else named_bar_sync(1 + team, P);
+        if (*reinterpret_cast<volatile int*>(abort_word) != 0) break;
+        if (tid == 0) {   // the row is in every thread's registers: refill the slot
+            cur->consumed += 1;
+            fence_proxy_async_smem();
+            issue();
+        }
+        if (++slot == nslot) {
+            slot = 0;
+            phase ^= 1;
+        }
+        float pp[TW];
+#pragma unroll
+        for (int i = 0; i < TW; ++i) pp[i] = part[pbuf * TW + i];
+        pbuf ^= 1;
+        const float inv = inv_rms_h(tree_sum_array<TW>(pp), fH, rH, pow2, a.eps);
+        const float2 inv2 = make_float2(inv, inv);
+        if (!has_line) continue;
+
+        uint32_t codes[8];
+        uint32_t sfw = 0u;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+            const uint4 w0 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk) * P + tid));
+            const uint4 w1 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk + 1) * P + tid));
+            const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t yw[8];
+            uint32_t m = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t xw = wv[8 * blk + i];
+                const float2 xg = GC0 ? mul_bf16x2_exact(xw, ws[i])
+                                      : mul2(unpack_bf16x2(xw), add2(gc2, unpack_bf16x2(ws[i])));
+                yw[i] = pack_bf16x2_rn(mul2(xg, inv2));
+                m = maxabs_bf16x2(m, yw[i]);
+            }
+            const float2 mf = unpack_bf16x2(m & 0x7fff7fffu);
+            const float amax = fmaxf(mf.x, mf.y);
+            const uint32_t sfc = cvt_e4m3_satfinite(__fmul_rn(gs, __fmul_rn(amax, kR6)));
+            const float sf_f = e4m3_to_f32(sfc);
+            const float os = (sf_f != 0.0f) ? __frcp_rn(__fmul_rn(sf_f, rgs)) : 0.0f;
+            const float2 os2 = make_float2(os, os);
+            float q[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 q2 = add2(mul2(unpack_bf16x2(yw[i]), os2), zero2);   // -0 -> +0
+                q[2 * i] = q2.x;
+                q[2 * i + 1] = q2.y;
+            }
+            codes[2 * blk] = cvt_e2m1x8(q);
+            codes[2 * blk + 1] = cvt_e2m1x8(q + 8);
+            sfw |= sfc << (8 * blk);
+        }
+        uint8_t* prow = a.packed + static_cast<size_t>(t) * (H / 2) + 32 * tid;
+        *reinterpret_cast<uint4*>(prow) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        *reinterpret_cast<uint4*>(prow + 16) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        *reinterpret_cast<uint32_t*>(a.sf + static_cast<size_t>(t) * nblocks + 4 * tid) = sfw;
+    }
+    if (tid == 0)
+        for (int f = cur->consumed; f < cur->issued; ++f)
+            mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+}
+
 namespace {
 
 template <int TW, bool SWZ, bool GC0>
@@ -233,6 +413,52 @@ cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a
     }
 }
 
+template <int TW, bool GC0>
+cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
+    constexpr int P = TW * 32;
+    constexpr int NTEAM = kConsumerThreads / P;
+    const int slot_bytes = slot_bytes_for(args.H);
+    WideLayout lay{NTEAM, 1, slot_bytes, P};
+    const size_t fixed = lay.total_bytes() - static_cast<size_t>(NTEAM) * slot_bytes;
+    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - 64 * NTEAM;
+    int nslot = avail / (NTEAM * slot_bytes);
+    if (nslot > 16) nslot = 16;
+    if (nslot < 2) return cudaErrorInvalidConfiguration;
+    lay.nslot = nslot;
+    NormQuantArgs a = args;
+    a.nslot = nslot;
+    const size_t smem = lay.total_bytes();
+    auto kern = norm_quant_wide_kernel<TW, GC0>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int grid = (a.M + NTEAM - 1) / NTEAM;
+    const int cap = device_info().sm_count;
+    if (grid > cap) grid = cap;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kConsumerThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, a);
+}
+
+template <bool GC0>
+cudaError_t launch_nq_wide_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
+    switch (TW) {
+        case 1: return launch_nq_wide<1, GC0>(tmap, a, s);
+        case 2: return launch_nq_wide<2, GC0>(tmap, a, s);
+        case 4: return launch_nq_wide<4, GC0>(tmap, a, s);
+        case 8: return launch_nq_wide<8, GC0>(tmap, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 // gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
 template <bool SWZ>
 cudaError_t launch_nq_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
@@ -261,8 +487,15 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
                      static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
     CUtensorMap tmap;
     if (swz && encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64),
-                               static_cast<uint32_t>(hs / 64)))
+                               static_cast<uint32_t>(hs / 64))) {
+        if (H >= 2048) {   // one 128-byte line per thread
+            int P = 32;
+            while (P < H / 64) P <<= 1;
+            return gc == 0.0f ? launch_nq_wide_tw<true>(P / 32, tmap, a, s)
+                              : launch_nq_wide_tw<false>(P / 32, tmap, a, s);
+        }
         return launch_nq_gc<true>(team_warps(H), tmap, a, s);
+    }
     std::memset(&tmap, 0, sizeof(tmap));
     return launch_nq_gc<false>(team_warps(H), tmap, a, s);
 }

@@ -78,6 +78,24 @@ __host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a *
 // Row slot size: the row's BF16 bytes, rounded up to the swizzle atom.
 __host__ __device__ inline int slot_bytes_for(int H) { return round_up(2 * H, kSlotAlign); }
 
+// Shared-memory carve-up of a wide-row CTA (one 128-byte line per thread):
+// row slots, the packed-weight table [8 chunks][P threads] x 16 B, slot
+// barriers, per-team partial buffers [2][TW], abort words and cursors.
+struct WideLayout {
+    int nteam, nslot, slot_bytes, P;
+    __host__ __device__ size_t slots_bytes() const { return static_cast<size_t>(nteam) * nslot * slot_bytes; }
+    __host__ __device__ size_t wtab_offset() const { return slots_bytes(); }              // [8][P] x 16 B
+    __host__ __device__ size_t bars_offset() const { return wtab_offset() + static_cast<size_t>(P) * 128; }
+    __host__ __device__ size_t part_offset() const {                                      // [nteam][2][TW] f32
+        return (bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t) + 15) & ~size_t(15);
+    }
+    __host__ __device__ size_t abort_offset() const { return part_offset() + static_cast<size_t>(nteam) * 2 * (P / 32) * sizeof(float); }
+    __host__ __device__ size_t cursor_offset() const { return abort_offset() + static_cast<size_t>(nteam) * 16; }
+    __host__ __device__ size_t total_bytes() const {
+        return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;
+    }
+};
+
 // Team-wide sum of one float per thread, in the canonical tree order.  One
 // named barrier per call when the team spans several warps.
 template <int TW>

@@ -9,11 +9,13 @@
 //   w_j   = s_{pick j} / (s_{pick 0} + ... + s_{pick k-1})   summed in pick order
 // and for an invalid token ids = -1, weights = 0 without reading its logits.
 //
-// Selection: every lane streams E/32 scores with 128-bit loads and keeps a
-// sorted register list of its best L candidates as 64-bit keys
-// (orderable(c) << 32 | ~id, so a larger key is the better pick and keys are
-// unique); k rounds of a warp-wide max over the lanes' list heads then emit
-// the picks in order.  Nothing is staged in shared or global scratch memory.
+// Selection: every lane reads E/32 scores with 128-bit loads and turns each
+// into a 32-bit order-preserving key; k merge rounds then emit the picks in
+// order, each a warp max (redux.sync) over the lanes' current bests with the
+// lowest expert id winning among equal keys (a warp min over the tied
+// lanes).  For E <= 512 a lane rescans its own <= 16 scores after a pick;
+// beyond that it keeps a sorted list of its best k.  Nothing is staged in
+// shared or global scratch memory.
 #include "common.cuh"
 #include "internal.h"
 
@@ -51,37 +53,154 @@ __device__ __forceinline__ float sigmoid_fixed(float x) {
     return __frcp_rn(__fadd_rn(1.0f, e));
 }
 
-// Key of expert e with selection score c: larger key = earlier pick.
-__device__ __forceinline__ uint64_t select_key(float c, int e) {
+// 32-bit selection key of a score: order-preserving image of the float
+// (larger key = larger score), -0 and +0 equal, NaN = 1 (below every number),
+// 0 = "no candidate".  Equal keys are broken by the lower expert id.
+__device__ __forceinline__ uint32_t score_key(float c) {
     c = __fadd_rn(c, 0.0f);                                  // -0 -> +0
     const uint32_t u = __float_as_uint(c);
-    uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    if (c != c) hi = 0u;                                     // NaN sorts last
-    return (static_cast<uint64_t>(hi) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
+    const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (c != c) ? 1u : k;
 }
 
-template <int L>
-__device__ __forceinline__ void list_insert(uint64_t (&list)[L], uint64_t key) {
-    if (key > list[L - 1]) {
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) { return __reduce_min_sync(0xffffffffu, v); }
+
+// One merge round: the warp's best (key, id) over every lane's best
+// candidate; returns true on the lane that owns it.
+__device__ __forceinline__ bool pick_round(uint32_t my_key, uint32_t my_id, uint32_t& key, uint32_t& id) {
+    key = warp_max_u32(my_key);
+    id = warp_min_u32(my_key == key ? my_id : 0xffffffffu);
+    return my_key == key && my_id == id;
+}
+
+// E <= 32 * EPL: every lane keeps its EPL scores (4 per 128-bit load, ids
+// 4 * (lane + 32 u) + i ascending with the register index) and rescans them
+// after each of its picks.
+template <int EPL>
+__device__ __forceinline__ void route_token_small(const float* l, const float* bias, int E, int k, int lane,
+                                                  bool vec, uint32_t& pick_key, uint32_t& pick_id) {
+    uint32_t key[EPL];
 #pragma unroll
-        for (int i = 0; i < L; ++i) {
-            const uint64_t hi = list[i] > key ? list[i] : key;
-            key = list[i] > key ? key : list[i];
-            list[i] = hi;
+    for (int u = 0; u < EPL / 4; ++u) {
+        const int q = lane + 32 * u;
+        if (vec && 4 * q + 3 < E) {
+            const float4 v = ld_nc_f4(l + 4 * q);
+            const float4 b = __ldg(reinterpret_cast<const float4*>(bias) + q);
+            key[4 * u + 0] = score_key(__fadd_rn(sigmoid_fixed(v.x), b.x));
+            key[4 * u + 1] = score_key(__fadd_rn(sigmoid_fixed(v.y), b.y));
+            key[4 * u + 2] = score_key(__fadd_rn(sigmoid_fixed(v.z), b.z));
+            key[4 * u + 3] = score_key(__fadd_rn(sigmoid_fixed(v.w), b.w));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = 4 * q + i;
+                key[4 * u + i] = e < E ? score_key(__fadd_rn(sigmoid_fixed(__ldg(l + e)), __ldg(bias + e))) : 0u;
+            }
+        }
+    }
+    // lane best: the largest key, lowest position among equals
+    auto best_of = [&](uint32_t& bk, int& bp) {
+        bk = 0u;
+        bp = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (key[i] > bk) {
+                bk = key[i];
+                bp = i;
+            }
+    };
+    uint32_t bk;
+    int bp;
+    best_of(bk, bp);
+    for (int j = 0; j < k; ++j) {
+        const uint32_t my_id = 4u * static_cast<uint32_t>(lane + 32 * (bp >> 2)) + static_cast<uint32_t>(bp & 3);
+        uint32_t key_j, id_j;
+        if (pick_round(bk, my_id, key_j, id_j)) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == bp) key[i] = 0u;
+            best_of(bk, bp);
+        }
+        if (lane == j) {
+            pick_key = key_j;
+            pick_id = id_j;
         }
     }
 }
 
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+// Larger E: every lane keeps a sorted list of its L best (key, id); ids arrive
+// in ascending order, so inserting strictly below equal keys keeps ties in id
+// order.
+template <int L>
+__device__ __forceinline__ void route_token_list(const float* l, const float* bias, int E, int k, int lane,
+                                                 bool vec, uint32_t& pick_key, uint32_t& pick_id) {
+    uint32_t lk[L], li[L];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
-        v = o > v ? o : v;
+    for (int i = 0; i < L; ++i) {
+        lk[i] = 0u;
+        li[i] = 0xffffffffu;
     }
-    return v;
+    auto insert = [&](uint32_t key, uint32_t id) {
+        if (key > lk[L - 1]) {
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const bool gt = key > lk[i];
+                const uint32_t tk = lk[i], ti = li[i];
+                lk[i] = gt ? key : tk;
+                li[i] = gt ? id : ti;
+                key = gt ? tk : key;
+                id = gt ? ti : id;
+            }
+        }
+    };
+    if (vec) {
+        const int nq = E >> 2;
+        for (int q0 = lane; q0 < nq; q0 += 128) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = q0 + 32 * u;
+                if (q < nq) v[u] = ld_nc_f4(l + 4 * q);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = q0 + 32 * u;
+                if (q < nq) {
+                    const float4 b = __ldg(reinterpret_cast<const float4*>(bias) + q);
+                    const uint32_t e = 4u * static_cast<uint32_t>(q);
+                    insert(score_key(__fadd_rn(sigmoid_fixed(v[u].x), b.x)), e);
+                    insert(score_key(__fadd_rn(sigmoid_fixed(v[u].y), b.y)), e + 1);
+                    insert(score_key(__fadd_rn(sigmoid_fixed(v[u].z), b.z)), e + 2);
+                    insert(score_key(__fadd_rn(sigmoid_fixed(v[u].w), b.w)), e + 3);
+                }
+            }
+        }
+    } else {
+        for (int e = lane; e < E; e += 32)
+            insert(score_key(__fadd_rn(sigmoid_fixed(__ldg(l + e)), __ldg(bias + e))), static_cast<uint32_t>(e));
+    }
+    for (int j = 0; j < k; ++j) {
+        uint32_t key_j, id_j;
+        if (pick_round(lk[0], li[0], key_j, id_j)) {
+#pragma unroll
+            for (int i = 0; i < L - 1; ++i) {
+                lk[i] = lk[i + 1];
+                li[i] = li[i + 1];
+            }
+            lk[L - 1] = 0u;
+            li[L - 1] = 0xffffffffu;
+        }
+        if (lane == j) {
+            pick_key = key_j;
+            pick_id = id_j;
+        }
+    }
 }
 
-template <int L>
+// MODE > 0: the small path with EPL = MODE scores per lane; MODE < 0: the
+// list path with L = -MODE entries.
+template <int MODE>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
                                                     const float* __restrict__ bias,
                                                     const uint8_t* __restrict__ mask, int T, int E,
@@ -105,49 +224,12 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             continue;
         }
         const float* l = logits + static_cast<size_t>(t) * E;
-        uint64_t list[L];
-#pragma unroll
-        for (int i = 0; i < L; ++i) list[i] = 0ull;
-
-        if (vec) {
-            const int nq = E >> 2;
-            for (int q0 = lane; q0 < nq; q0 += 128) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int q = q0 + 32 * u;
-                    if (q < nq) v[u] = ld_nc_f4(l + 4 * q);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int q = q0 + 32 * u;
-                    if (q < nq) {
-                        const float4 b = __ldg(reinterpret_cast<const float4*>(bias) + q);
-                        const int e = 4 * q;
-                        list_insert<L>(list, select_key(__fadd_rn(sigmoid_fixed(v[u].x), b.x), e));
-                        list_insert<L>(list, select_key(__fadd_rn(sigmoid_fixed(v[u].y), b.y), e + 1));
-                        list_insert<L>(list, select_key(__fadd_rn(sigmoid_fixed(v[u].z), b.z), e + 2));
-                        list_insert<L>(list, select_key(__fadd_rn(sigmoid_fixed(v[u].w), b.w), e + 3));
-                    }
-                }
-            }
-        } else {
-            for (int e = lane; e < E; e += 32)
-                list_insert<L>(list, select_key(__fadd_rn(sigmoid_fixed(__ldg(l + e)), __ldg(bias + e)), e));
-        }
-
-        // k rounds: the lane holding the best remaining head pops it.
-        uint64_t mine = 0ull;
-        for (int j = 0; j < k; ++j) {
-            const uint64_t best = warp_max_u64(list[0]);
-            if (list[0] == best) {
-#pragma unroll
-                for (int i = 0; i < L - 1; ++i) list[i] = list[i + 1];
-                list[L - 1] = 0ull;
-            }
-            if (lane == j) mine = best;
-        }
-        const int e = static_cast<int>(~static_cast<uint32_t>(mine));
+        uint32_t pick_key = 0u, pick_id = 0u;
+        if constexpr (MODE > 0)
+            route_token_small<MODE>(l, bias, E, k, lane, vec, pick_key, pick_id);
+        else
+            route_token_list<-MODE>(l, bias, E, k, lane, vec, pick_key, pick_id);
+        const int e = static_cast<int>(pick_id);
         float s = 0.0f;
         if (lane < k) s = sigmoid_fixed(__ldg(l + e));
         float S = 0.0f;
@@ -162,7 +244,6 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                          int k, int32_t* ids, float* weights, cudaStream_t s) {
     const int per_lane = (E + 31) / 32;
-    const int need = per_lane < k ? per_lane : k;
     const int warps_per_cta = 8;
     int grid = (T + warps_per_cta - 1) / warps_per_cta;
     const int cap = device_info().sm_count * 8;
@@ -176,9 +257,14 @@ cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (need <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8>, logits, bias, mask, T, E, k, ids, weights);
-    if (need <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16>, logits, bias, mask, T, E, k, ids, weights);
-    return cudaLaunchKernelEx(&cfg, route_kernel<32>, logits, bias, mask, T, E, k, ids, weights);
+    // scores per lane, rounded up to whole 128-bit loads
+    const int epl = (per_lane + 3) / 4 * 4;
+    if (epl <= 4) return cudaLaunchKernelEx(&cfg, route_kernel<4>, logits, bias, mask, T, E, k, ids, weights);
+    if (epl <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8>, logits, bias, mask, T, E, k, ids, weights);
+    if (epl <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16>, logits, bias, mask, T, E, k, ids, weights);
+    if (k <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<-8>, logits, bias, mask, T, E, k, ids, weights);
+    if (k <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<-16>, logits, bias, mask, T, E, k, ids, weights);
+    return cudaLaunchKernelEx(&cfg, route_kernel<-32>, logits, bias, mask, T, E, k, ids, weights);
 }
 
 }  // namespace mb
