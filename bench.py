@@ -325,8 +325,7 @@ def run_ours(args, world, rank, local):
                          "bytes_per_launch": cmb_bytes_net,
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},
-            "stages_ms": {"route": stage_ms[0], "norm_quant": stage_ms[1],
-                          "combine": stage_ms[2]},
+            "stages_ms": {"route": stage_ms[0], "norm_quant": stage_ms[1], "combine": stage_ms[2]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,

@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     STAGE_JOIN,
     STAGE_NORM_QUANT,
     STAGE_ROUTE,
+    STAGE_ROUTE_NORM_QUANT,
     device_status,
     expert_combine,
     expert_combine_join,
@@ -23,6 +24,7 @@ from ._lib import (  # noqa: F401
     lib_path,
     load,
     moe_route,
+    moe_route_norm_quant,
     norm_quant_nvfp4,
     residual_join,
     supported,

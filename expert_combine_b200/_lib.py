@@ -15,6 +15,7 @@ STAGE_NORM_QUANT = 1
 STAGE_COMBINE = 2
 STAGE_JOIN = 3
 STAGE_COMBINE_JOIN = 4
+STAGE_ROUTE_NORM_QUANT = 5
 
 _lock = threading.Lock()
 _lib = None
@@ -57,6 +58,8 @@ def load() -> ctypes.CDLL:
                 "residual_join": [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32, P],
                 "expert_combine_join": [P, i64, i32, P, P, i32, i32, P, f32, f32, P, P, P, f32, f32,
                                         f32, P, f32, f32, P, P],
+                "moe_route_norm_quant": [P, P, P, i32, i32, P, P, P, i32, i32, i32, P, f32, f32, P, P,
+                                         P, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
                 "mb_last_error": [],
                 "mb_device_status": [],
@@ -159,6 +162,47 @@ def norm_quant_nvfp4(x: torch.Tensor, num_tokens: int, norm_w: torch.Tensor, gai
            load().norm_quant_nvfp4(_ptr(x), M, H, tp, _ptr(norm_w), float(gain_center), float(eps),
                                    _ptr(global_scale), _ptr(packed), _ptr(sf), _stream(stream)))
     return packed, sf
+
+
+def moe_route_norm_quant(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor, k: int,
+                         x: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
+                         global_scale: torch.Tensor, tp: int = 1,
+                         topk_ids: Optional[torch.Tensor] = None,
+                         topk_weights: Optional[torch.Tensor] = None,
+                         packed: Optional[torch.Tensor] = None, sf: Optional[torch.Tensor] = None,
+                         stream=None):
+    """Router gate and RMSNorm + NVFP4 of the same tokens in one launch.
+
+    -> (topk_ids, topk_weights, packed, sf), equal to moe_route + norm_quant_nvfp4.
+    """
+    _want(logits, torch.float32, "logits")
+    _want(bias, torch.float32, "bias")
+    _want(token_mask, torch.uint8, "token_mask")
+    _want(x, torch.bfloat16, "x")
+    _want(norm_w, torch.bfloat16, "norm_w")
+    _want(global_scale, torch.float32, "global_scale")
+    T, E = logits.shape
+    H = norm_w.numel()
+    if x.numel() != T * H or bias.numel() != E or token_mask.numel() != T:
+        raise ValueError("moe_route_norm_quant: shape mismatch")
+    dev = logits.device
+    if topk_ids is None:
+        topk_ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if topk_weights is None:
+        topk_weights = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if packed is None:
+        packed = torch.empty(T, H // 2, dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(T, H // 16, dtype=torch.uint8, device=dev)
+    for t, dt, name in ((topk_ids, torch.int32, "topk_ids"), (topk_weights, torch.float32, "topk_weights"),
+                        (packed, torch.uint8, "packed"), (sf, torch.uint8, "sf")):
+        _want(t, dt, name)
+    _check("moe_route_norm_quant",
+           load().moe_route_norm_quant(_ptr(logits), _ptr(bias), _ptr(token_mask), E, k,
+                                       _ptr(topk_ids), _ptr(topk_weights), _ptr(x), T, H, tp,
+                                       _ptr(norm_w), float(gain_center), float(eps),
+                                       _ptr(global_scale), _ptr(packed), _ptr(sf), _stream(stream)))
+    return topk_ids, topk_weights, packed, sf
 
 
 def expert_combine(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,

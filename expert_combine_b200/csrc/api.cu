@@ -71,23 +71,52 @@ int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp) {
             return (hidden_ok(H) && k >= 1 && k <= kMaxTopK) ? 1 : 0;
         case MB_STAGE_JOIN:
             return hidden_ok(H) ? 1 : 0;
+        case MB_STAGE_ROUTE_NORM_QUANT:
+            return (moe_boundary_supported(MB_STAGE_ROUTE, T, H, E, k, tp) &&
+                    moe_boundary_supported(MB_STAGE_NORM_QUANT, T, H, E, k, tp))
+                       ? 1
+                       : 0;
         default:
             return 0;
     }
 }
 
-int moe_route(const float* logits, const float* bias, const uint8_t* token_mask, int T, int E, int k,
-              int32_t* topk_ids, float* topk_weights, void* stream) {
-    if (T < 0 || E < 0 || k < 0) return fail(MB_ERR_INVALID_ARG, "moe_route: negative size");
+static int check_route(const char* fn, const float* logits, const float* bias, const uint8_t* token_mask,
+                       int T, int E, int k, int32_t* topk_ids, float* topk_weights) {
+    if (T < 0 || E < 0 || k < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
     if (!moe_boundary_supported(MB_STAGE_ROUTE, T, 0, E, k, 1))
-        return fail(MB_ERR_UNSUPPORTED, "moe_route: needs 1 <= k <= %d and k <= E <= %d (k=%d, E=%d)",
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs 1 <= k <= %d and k <= E <= %d (k=%d, E=%d)", fn,
                     kMaxTopK, kMaxExperts, k, E);
     if (T == 0) return MB_OK;
     if (!logits || !bias || !token_mask || !topk_ids || !topk_weights)
-        return fail(MB_ERR_INVALID_ARG, "moe_route: null pointer");
+        return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
     if (!aligned16(logits) || !aligned16(bias) || !aligned16(token_mask) || !aligned16(topk_ids) ||
         !aligned16(topk_weights))
-        return fail(MB_ERR_INVALID_ARG, "moe_route: pointers must be 16-byte aligned");
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return MB_OK;
+}
+
+static int check_norm_quant(const char* fn, const uint16_t* x, int M, int H, int tp, const uint16_t* norm_w,
+                            const float* global_scale, uint8_t* packed, uint8_t* sf) {
+    if (M < 0 || H < 0 || tp < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (tp == 0 || H % 16 != 0 || H % tp != 0 || (H / tp) % 16 != 0)
+        return fail(MB_ERR_INVALID_ARG,
+                    "%s: needs H %% 16 == 0, tp >= 1, H %% tp == 0, (H/tp) %% 16 == 0 (H=%d, tp=%d)", fn, H,
+                    tp);
+    if (!moe_boundary_supported(MB_STAGE_NORM_QUANT, M, H, 0, 0, tp))
+        return fail(MB_ERR_UNSUPPORTED, "%s: H=%d outside 16..%d", fn, H, kMaxHidden);
+    if (M == 0) return MB_OK;
+    if (!x || !norm_w || !global_scale || !packed || !sf) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(x) || !aligned16(norm_w) || !aligned16(packed) || !aligned16(sf) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return MB_OK;
+}
+
+int moe_route(const float* logits, const float* bias, const uint8_t* token_mask, int T, int E, int k,
+              int32_t* topk_ids, float* topk_weights, void* stream) {
+    const int st = check_route("moe_route", logits, bias, token_mask, T, E, k, topk_ids, topk_weights);
+    if (st != MB_OK || T == 0) return st;
     return cuda_status(launch_route(logits, bias, token_mask, T, E, k, topk_ids, topk_weights,
                                     static_cast<cudaStream_t>(stream)),
                        "moe_route");
@@ -95,22 +124,25 @@ int moe_route(const float* logits, const float* bias, const uint8_t* token_mask,
 
 int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* norm_w, float gain_center,
                      float eps, const float* global_scale, uint8_t* packed, uint8_t* sf, void* stream) {
-    if (M < 0 || H < 0 || tp < 0) return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: negative size");
-    if (tp == 0 || H % 16 != 0 || H % tp != 0 || (H / tp) % 16 != 0)
-        return fail(MB_ERR_INVALID_ARG,
-                    "norm_quant_nvfp4: needs H %% 16 == 0, tp >= 1, H %% tp == 0, (H/tp) %% 16 == 0 "
-                    "(H=%d, tp=%d)", H, tp);
-    if (!moe_boundary_supported(MB_STAGE_NORM_QUANT, M, H, 0, 0, tp))
-        return fail(MB_ERR_UNSUPPORTED, "norm_quant_nvfp4: H=%d outside 16..%d", H, kMaxHidden);
-    if (M == 0) return MB_OK;
-    if (!x || !norm_w || !global_scale || !packed || !sf)
-        return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: null pointer");
-    if (!aligned16(x) || !aligned16(norm_w) || !aligned16(packed) || !aligned16(sf) ||
-        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
-        return fail(MB_ERR_INVALID_ARG, "norm_quant_nvfp4: pointers must be 16-byte aligned");
+    const int st = check_norm_quant("norm_quant_nvfp4", x, M, H, tp, norm_w, global_scale, packed, sf);
+    if (st != MB_OK || M == 0) return st;
     return cuda_status(launch_norm_quant(x, M, H, tp, norm_w, gain_center, eps, global_scale, packed, sf,
                                          static_cast<cudaStream_t>(stream)),
                        "norm_quant_nvfp4");
+}
+
+int moe_route_norm_quant(const float* logits, const float* bias, const uint8_t* token_mask, int E, int k,
+                         int32_t* topk_ids, float* topk_weights, const uint16_t* x, int M, int H, int tp,
+                         const uint16_t* norm_w, float gain_center, float eps, const float* global_scale,
+                         uint8_t* packed, uint8_t* sf, void* stream) {
+    int st = check_route("moe_route_norm_quant", logits, bias, token_mask, M, E, k, topk_ids, topk_weights);
+    if (st != MB_OK) return st;
+    st = check_norm_quant("moe_route_norm_quant", x, M, H, tp, norm_w, global_scale, packed, sf);
+    if (st != MB_OK || M == 0) return st;
+    return cuda_status(launch_route_norm_quant(logits, bias, token_mask, E, k, topk_ids, topk_weights, x, M, H,
+                                               tp, norm_w, gain_center, eps, global_scale, packed, sf,
+                                               static_cast<cudaStream_t>(stream)),
+                       "moe_route_norm_quant");
 }
 
 static int check_combine(const char* fn, const uint16_t* expert_out, int64_t num_rows, int H,

@@ -20,6 +20,11 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
                               float eps, const float* gs, uint8_t* packed, uint8_t* sf,
                               cudaStream_t s);
 
+cudaError_t launch_route_norm_quant(const float* logits, const float* bias, const uint8_t* mask, int E, int k,
+                                    int32_t* ids, float* weights, const uint16_t* x, int M, int H, int tp,
+                                    const uint16_t* w, float gc, float eps, const float* gs, uint8_t* packed,
+                                    uint8_t* sf, cudaStream_t s);
+
 struct JoinArgs {
     float* residual;            // [T, H] FP32 in/out; NULL = no join
     const uint16_t* gain;       // [H] BF16

@@ -4,5 +4,5 @@
 // library is compiled as one unit instead of relocatable device code.
 #include "api.cu"
 #include "combine.cu"
-#include "norm_quant.cu"
 #include "route.cu"
+#include "norm_quant.cu"

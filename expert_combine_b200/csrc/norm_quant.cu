@@ -27,6 +27,13 @@ struct NormQuantArgs {
     uint8_t* packed;
     uint8_t* sf;
     int nslot;
+    // router gate fused into the wide kernel (RMODE > 0): the same M tokens
+    const float* logits;
+    const float* bias;
+    const uint8_t* mask;
+    int E, k;
+    int32_t* ids;
+    float* weights;
 };
 
 template <int TW, bool SWZ, bool GC0>
@@ -194,7 +201,12 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // keeps its 32 words in registers across the team barrier, so the slot is
 // refilled as soon as the barrier has passed.  The packed BF16 weights sit in
 // a shared-memory table read without bank conflicts.
-template <int TW, bool GC0>
+//
+// With RMODE > 0 the kernel also runs the router gate for its tokens (the two
+// pre-expert stages are independent): for the team's i-th token, warp
+// i % TW of the team loads the token's logits before the norm passes and
+// selects its top-k after them (RMODE scores per lane, E <= 32 * RMODE).
+template <int TW, bool GC0, int RMODE>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     norm_quant_wide_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
     constexpr int P = TW * 32;
@@ -277,8 +289,17 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int sw = tid & 7;
     const int nblocks = H / 16;
 
-    int slot = 0, phase = 0, pbuf = 0;
-    for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride) {
+    int slot = 0, phase = 0, pbuf = 0, iter = 0;
+    constexpr int NL = RMODE > 0 ? RMODE : 4;
+    for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride, ++iter) {
+        // router: this warp's token?  issue its logit loads before the norm work
+        const bool router = RMODE > 0 && (iter % TW) == warp_in_team;
+        const bool route_valid = router && a.mask[t] != 0;
+        float lv[NL];
+        if constexpr (RMODE > 0) {
+            if (route_valid)
+                load_logits<NL>(a.logits + static_cast<size_t>(t) * a.E, a.E, lane, (a.E & 3) == 0, lv);
+        }
         const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
         uint32_t wv[32];
         float b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -322,8 +343,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         pbuf ^= 1;
         const float inv = inv_rms_h(tree_sum_array<TW>(pp), fH, rH, pow2, a.eps);
         const float2 inv2 = make_float2(inv, inv);
-        if (!has_line) continue;
-
+        if (has_line) {
         uint32_t codes[8];
         uint32_t sfw = 0u;
 #pragma unroll
@@ -362,6 +382,23 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         *reinterpret_cast<uint4*>(prow) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
         *reinterpret_cast<uint4*>(prow + 16) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
         *reinterpret_cast<uint32_t*>(a.sf + static_cast<size_t>(t) * nblocks + 4 * tid) = sfw;
+        }
+        if constexpr (RMODE > 0) {
+            if (router) {
+                int32_t* id_row = a.ids + static_cast<size_t>(t) * a.k;
+                float* w_row = a.weights + static_cast<size_t>(t) * a.k;
+                if (!route_valid) {
+                    if (lane < a.k) {
+                        id_row[lane] = -1;
+                        w_row[lane] = 0.0f;
+                    }
+                } else {
+                    uint32_t pick_key = 0u, pick_id = 0u;
+                    select_small<NL>(lv, a.bias, a.E, a.k, lane, (a.E & 3) == 0, pick_key, pick_id);
+                    route_write(a.logits + static_cast<size_t>(t) * a.E, a.k, lane, pick_id, id_row, w_row);
+                }
+            }
+        }
     }
     if (tid == 0)
         for (int f = cur->consumed; f < cur->issued; ++f)
@@ -413,7 +450,7 @@ cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a
     }
 }
 
-template <int TW, bool GC0>
+template <int TW, bool GC0, int RMODE>
 cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
     constexpr int P = TW * 32;
     constexpr int NTEAM = kConsumerThreads / P;
@@ -428,7 +465,7 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     NormQuantArgs a = args;
     a.nslot = nslot;
     const size_t smem = lay.total_bytes();
-    auto kern = norm_quant_wide_kernel<TW, GC0>;
+    auto kern = norm_quant_wide_kernel<TW, GC0, RMODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -448,15 +485,21 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     return cudaLaunchKernelEx(&cfg, kern, tmap, a);
 }
 
-template <bool GC0>
+template <bool GC0, int RMODE>
 cudaError_t launch_nq_wide_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
     switch (TW) {
-        case 1: return launch_nq_wide<1, GC0>(tmap, a, s);
-        case 2: return launch_nq_wide<2, GC0>(tmap, a, s);
-        case 4: return launch_nq_wide<4, GC0>(tmap, a, s);
-        case 8: return launch_nq_wide<8, GC0>(tmap, a, s);
+        case 1: return launch_nq_wide<1, GC0, RMODE>(tmap, a, s);
+        case 2: return launch_nq_wide<2, GC0, RMODE>(tmap, a, s);
+        case 4: return launch_nq_wide<4, GC0, RMODE>(tmap, a, s);
+        case 8: return launch_nq_wide<8, GC0, RMODE>(tmap, a, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <int RMODE>
+cudaError_t launch_nq_wide_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
+    return a.gc == 0.0f ? launch_nq_wide_tw<true, RMODE>(TW, tmap, a, s)
+                        : launch_nq_wide_tw<false, RMODE>(TW, tmap, a, s);
 }
 
 // gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
@@ -477,27 +520,60 @@ int team_warps(int H) {
     return P / 32;
 }
 
+namespace {
+
+// Tensor map and team width of the norm-quant row copies; false when the
+// wide tensor-map path does not apply.
+bool wide_nq_plan(const uint16_t* x, int M, int H, int tp, CUtensorMap& tmap, int& TW) {
+    const int hs = H / tp;
+    const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
+                     static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
+    if (!swz || H < 2048) return false;
+    if (!encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64), static_cast<uint32_t>(hs / 64)))
+        return false;
+    int P = 32;
+    while (P < H / 64) P <<= 1;
+    TW = P / 32;
+    return true;
+}
+
+}  // namespace
+
 cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uint16_t* w, float gc,
                               float eps, const float* gs, uint8_t* packed, uint8_t* sf,
                               cudaStream_t s) {
-    const NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
+    NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
+    CUtensorMap tmap;
+    int TW = 0;
+    if (wide_nq_plan(x, M, H, tp, tmap, TW)) return launch_nq_wide_gc<0>(TW, tmap, a, s);
     const int hs = H / tp;
-    // the tensor path needs 64-element lines and each segment on a swizzle atom
     const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
                      static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
-    CUtensorMap tmap;
     if (swz && encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64),
-                               static_cast<uint32_t>(hs / 64))) {
-        if (H >= 2048) {   // one 128-byte line per thread
-            int P = 32;
-            while (P < H / 64) P <<= 1;
-            return gc == 0.0f ? launch_nq_wide_tw<true>(P / 32, tmap, a, s)
-                              : launch_nq_wide_tw<false>(P / 32, tmap, a, s);
-        }
+                               static_cast<uint32_t>(hs / 64)))
         return launch_nq_gc<true>(team_warps(H), tmap, a, s);
-    }
     std::memset(&tmap, 0, sizeof(tmap));
     return launch_nq_gc<false>(team_warps(H), tmap, a, s);
+}
+
+cudaError_t launch_route_norm_quant(const float* logits, const float* bias, const uint8_t* mask, int E, int k,
+                                    int32_t* ids, float* weights, const uint16_t* x, int M, int H, int tp,
+                                    const uint16_t* w, float gc, float eps, const float* gs, uint8_t* packed,
+                                    uint8_t* sf, cudaStream_t s) {
+    NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0, logits, bias, mask, E, k, ids, weights};
+    CUtensorMap tmap;
+    int TW = 0;
+    const int per_lane = (E + 31) / 32;
+    const int epl = (per_lane + 3) / 4 * 4;
+    if (epl <= 16 && wide_nq_plan(x, M, H, tp, tmap, TW)) {
+        if (epl <= 4) return launch_nq_wide_gc<4>(TW, tmap, a, s);
+        if (epl <= 8) return launch_nq_wide_gc<8>(TW, tmap, a, s);
+        return launch_nq_wide_gc<16>(TW, tmap, a, s);
+    }
+    // shapes the fused kernel does not take: the two kernels back to back
+    cudaError_t e = launch_route(logits, bias, mask, M, E, k, ids, weights, s);
+    if (e != cudaSuccess) return e;
+    return launch_norm_quant(x, M, H, tp, w, gc, eps, gs, packed, sf, s);
 }
 
 }  // namespace mb

@@ -74,28 +74,46 @@ __device__ __forceinline__ bool pick_round(uint32_t my_key, uint32_t my_id, uint
     return my_key == key && my_id == id;
 }
 
-// E <= 32 * EPL: every lane keeps its EPL scores (4 per 128-bit load, ids
-// 4 * (lane + 32 u) + i ascending with the register index) and rescans them
-// after each of its picks.
+// This lane's EPL logits of a token row (4 per 128-bit load, ids
+// 4 * (lane + 32 u) + i ascending with the register index; 0 past E).
 template <int EPL>
-__device__ __forceinline__ void route_token_small(const float* l, const float* bias, int E, int k, int lane,
-                                                  bool vec, uint32_t& pick_key, uint32_t& pick_id) {
-    uint32_t key[EPL];
+__device__ __forceinline__ void load_logits(const float* l, int E, int lane, bool vec, float (&lv)[EPL]) {
 #pragma unroll
     for (int u = 0; u < EPL / 4; ++u) {
         const int q = lane + 32 * u;
         if (vec && 4 * q + 3 < E) {
             const float4 v = ld_nc_f4(l + 4 * q);
+            lv[4 * u + 0] = v.x;
+            lv[4 * u + 1] = v.y;
+            lv[4 * u + 2] = v.z;
+            lv[4 * u + 3] = v.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) lv[4 * u + i] = (4 * q + i < E) ? __ldg(l + 4 * q + i) : 0.0f;
+        }
+    }
+}
+
+// E <= 32 * EPL: every lane keeps its EPL scores and rescans them after each
+// of its picks.
+template <int EPL>
+__device__ __forceinline__ void select_small(const float (&lv)[EPL], const float* bias, int E, int k, int lane,
+                                             bool vec, uint32_t& pick_key, uint32_t& pick_id) {
+    uint32_t key[EPL];
+#pragma unroll
+    for (int u = 0; u < EPL / 4; ++u) {
+        const int q = lane + 32 * u;
+        if (vec && 4 * q + 3 < E) {
             const float4 b = __ldg(reinterpret_cast<const float4*>(bias) + q);
-            key[4 * u + 0] = score_key(__fadd_rn(sigmoid_fixed(v.x), b.x));
-            key[4 * u + 1] = score_key(__fadd_rn(sigmoid_fixed(v.y), b.y));
-            key[4 * u + 2] = score_key(__fadd_rn(sigmoid_fixed(v.z), b.z));
-            key[4 * u + 3] = score_key(__fadd_rn(sigmoid_fixed(v.w), b.w));
+            key[4 * u + 0] = score_key(__fadd_rn(sigmoid_fixed(lv[4 * u + 0]), b.x));
+            key[4 * u + 1] = score_key(__fadd_rn(sigmoid_fixed(lv[4 * u + 1]), b.y));
+            key[4 * u + 2] = score_key(__fadd_rn(sigmoid_fixed(lv[4 * u + 2]), b.z));
+            key[4 * u + 3] = score_key(__fadd_rn(sigmoid_fixed(lv[4 * u + 3]), b.w));
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int e = 4 * q + i;
-                key[4 * u + i] = e < E ? score_key(__fadd_rn(sigmoid_fixed(__ldg(l + e)), __ldg(bias + e))) : 0u;
+                key[4 * u + i] = e < E ? score_key(__fadd_rn(sigmoid_fixed(lv[4 * u + i]), __ldg(bias + e))) : 0u;
             }
         }
     }
@@ -126,6 +144,21 @@ __device__ __forceinline__ void route_token_small(const float* l, const float* b
             pick_key = key_j;
             pick_id = id_j;
         }
+    }
+}
+
+// The picks' unbiased sigmoids, renormalised in pick order (lane j < k holds
+// pick j), written with the ids.
+__device__ __forceinline__ void route_write(const float* l, int k, int lane, uint32_t pick_id, int32_t* id_row,
+                                            float* w_row) {
+    const int e = static_cast<int>(pick_id);
+    float s = 0.0f;
+    if (lane < k) s = sigmoid_fixed(__ldg(l + e));
+    float S = 0.0f;
+    for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, s, j));
+    if (lane < k) {
+        id_row[lane] = e;
+        w_row[lane] = __fdiv_rn(s, S);
     }
 }
 
@@ -225,19 +258,14 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
         }
         const float* l = logits + static_cast<size_t>(t) * E;
         uint32_t pick_key = 0u, pick_id = 0u;
-        if constexpr (MODE > 0)
-            route_token_small<MODE>(l, bias, E, k, lane, vec, pick_key, pick_id);
-        else
+        if constexpr (MODE > 0) {
+            float lv[MODE];
+            load_logits<MODE>(l, E, lane, vec, lv);
+            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+        } else {
             route_token_list<-MODE>(l, bias, E, k, lane, vec, pick_key, pick_id);
-        const int e = static_cast<int>(pick_id);
-        float s = 0.0f;
-        if (lane < k) s = sigmoid_fixed(__ldg(l + e));
-        float S = 0.0f;
-        for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, s, j));
-        if (lane < k) {
-            id_row[lane] = e;
-            w_row[lane] = __fdiv_rn(s, S);
         }
+        route_write(l, k, lane, pick_id, id_row, w_row);
     }
 }
 

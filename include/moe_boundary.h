@@ -92,6 +92,25 @@ int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* no
                      uint8_t* sf, void* stream);
 
 /*
+ * moe_route_norm_quant -- moe_route and norm_quant_nvfp4 of the same M tokens
+ * in one launch.
+ *
+ * Source: as moe_route and norm_quant_nvfp4.  The two pre-expert stages read
+ * disjoint inputs and are independent; TensorRT-LLM PR 21356 ("Where they
+ * plug in") runs the pre-expert norm on an auxiliary stream while the router
+ * runs on the current one.  Here one kernel does both: the team that
+ * normalises and quantises token t also routes it.  Arguments and results
+ * are those of the two calls with T = M, bit for bit.  When the fused kernel
+ * does not take the sizes (E > 512, H < 2048, H % 64 != 0, or a rank-block
+ * shard not a multiple of 512) the two kernels run back to back on `stream`.
+ * Supported: the union of both calls' rules.
+ */
+int moe_route_norm_quant(const float* logits, const float* bias, const uint8_t* token_mask, int E, int k,
+                         int32_t* topk_ids, float* topk_weights, const uint16_t* x, int M, int H, int tp,
+                         const uint16_t* norm_w, float gain_center, float eps, const float* global_scale,
+                         uint8_t* packed, uint8_t* sf, void* stream);
+
+/*
  * expert_combine -- post-expert RMSNorm of each selected row + weighted sum.
  *
  * Source: TensorRT-LLM PR 21356, description, "Post-expert norm and combine"
@@ -167,6 +186,7 @@ enum {
     MB_STAGE_COMBINE = 2,
     MB_STAGE_JOIN = 3,
     MB_STAGE_COMBINE_JOIN = 4,
+    MB_STAGE_ROUTE_NORM_QUANT = 5,
 };
 
 /*

@@ -36,6 +36,25 @@ def test_route_shapes(cuda_dev, E, k):
     check_route(case)
 
 
+@pytest.mark.parametrize("T,H,E,k,tp", [(37, 8192, 256, 8, 1), (64, 4096, 512, 22, 4), (19, 2048, 100, 7, 1),
+                                        (40, 2688, 128, 8, 1), (16, 1024, 256, 8, 1),
+                                        (24, 4096, 2560, 8, 4), (9, 16384, 512, 32, 1)])
+def test_route_norm_quant_fused(cuda_dev, T, H, E, k, tp):
+    """One launch (or the two kernels where the fused one does not apply) equals both stages."""
+    case = synth.make_case("tiny", device=cuda_dev, T=T, H=H, E=E, k=k, tp=tp, join=False)
+    ids, w, packed, sf = eb.moe_route_norm_quant(case.logits, case.bias, case.mask, case.k, case.x,
+                                                 case.norm_w, case.gc, case.eps, case.gs, tp=tp)
+    torch.cuda.synchronize()
+    ids_o, w_o = oracle.route(synth.host(case.logits), synth.host(case.bias), synth.host(case.mask),
+                              case.k)
+    assert np.array_equal(synth.host(ids), ids_o)
+    assert np.array_equal(synth.host(w).view(np.uint32), w_o.view(np.uint32))
+    p_o, s_o = oracle.norm_quant(synth.host(case.x), case.T, case.H, tp, synth.host(case.norm_w),
+                                 case.gc, case.eps, float(synth.host(case.gs)[0]))
+    assert np.array_equal(synth.host(packed), p_o) and np.array_equal(synth.host(sf), s_o)
+    assert eb.device_status() == 0
+
+
 def test_route_integer_logits_many_ties(cuda_dev):
     g = torch.Generator(device=cuda_dev)
     g.manual_seed(5)
