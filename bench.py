@@ -4,7 +4,9 @@
 Workload (one step, per GPU): T=8192 tokens, H=8192, E=256 experts, top-8,
 router logits FP32 N(0, 2), 5% of tokens masked, 1% of expert slots invalid,
 expert outputs [T*8, H] BF16 -- synthetic, seeded, resident in HBM.  The
-three calls go through the library's C ABI on one stream.
+three calls go through the library's C ABI on one stream (moe_route,
+norm_quant_nvfp4, expert_combine; `--joint` enqueues the first two with the
+single moe_route_norm_quant call).
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -239,21 +241,28 @@ def run_ours(args, world, rank, local):
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def pre_expert():
+        # the router gate and the pre-expert RMSNorm + NVFP4 of the same tokens
+        if not args.joint:
+            eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+            eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
+                                sf=sf)
+        else:
+            eb.moe_route_norm_quant(case.logits, case.bias, case.mask, k, case.x, case.norm_w,
+                                    case.gc, case.eps, case.gs, topk_ids=ids, topk_weights=w,
+                                    packed=packed, sf=sf)
+
     def step(ev=None):
-        # ev: 4 events bracketing the three launches (stage times on this stream)
+        # ev: 3 events bracketing the pre-expert stages and the combine
         if ev is not None:
             ev[0].record(stream)
-        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+        pre_expert()
         if ev is not None:
             ev[1].record(stream)
-        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
-                            sf=sf)
-        if ev is not None:
-            ev[2].record(stream)
         eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                           case.eps, out=out)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -261,7 +270,7 @@ def run_ours(args, world, rank, local):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
@@ -272,9 +281,9 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     barrier(world)
-    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(3)]
-    combine_ms = stage_ms[2]
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(2)]
+    combine_ms = stage_ms[1]
     step_ms_max = max_over_ranks(step_ms, world)
     ms_per_step = step_ms_max / args.steps
 
@@ -291,7 +300,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the same calls with host buffers (pinned), copies inside
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
-                                           steps=max(2, min(args.steps, 5)))
+                                           pre_expert, steps=max(2, min(args.steps, 5)))
 
     tokens_per_s = T * world / (ms_per_step * 1e-3)
     result = None
@@ -325,7 +334,7 @@ def run_ours(args, world, rank, local):
                          "bytes_per_launch": cmb_bytes_net,
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},
-            "stages_ms": {"route": stage_ms[0], "norm_quant": stage_ms[1], "combine": stage_ms[2]},
+            "stages_ms": {"route_norm_quant": stage_ms[0], "combine": stage_ms[1]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,
@@ -339,7 +348,7 @@ def run_ours(args, world, rank, local):
     return result
 
 
-def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps):
+def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, pre_expert, steps):
     """Host inputs (pinned) -> device -> the three calls -> host outputs, per step."""
     T, H, k = case.T, case.H, case.k
     h_in = {name: t.detach().cpu().pin_memory() for name, t in
@@ -355,9 +364,7 @@ def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, steps):
     def one():
         for name, h in h_in.items():
             d_in[name].copy_(h, non_blocking=True)
-        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
-        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
-                            sf=sf)
+        pre_expert()
         eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                           case.eps, out=out)
         for name, d in (("ids", ids), ("w", w), ("packed", packed), ("sf", sf), ("out", out)):
@@ -384,6 +391,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default: the workload's 8192); smaller for profiling")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--joint", action="store_true",
+                    help="enqueue the pre-expert stages with the joint moe_route_norm_quant call")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -27,13 +27,6 @@ struct NormQuantArgs {
     uint8_t* packed;
     uint8_t* sf;
     int nslot;
-    // router gate fused into the wide kernel (RMODE > 0): the same M tokens
-    const float* logits;
-    const float* bias;
-    const uint8_t* mask;
-    int E, k;
-    int32_t* ids;
-    float* weights;
 };
 
 template <int TW, bool SWZ, bool GC0>
@@ -201,12 +194,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // keeps its 32 words in registers across the team barrier, so the slot is
 // refilled as soon as the barrier has passed.  The packed BF16 weights sit in
 // a shared-memory table read without bank conflicts.
-//
-// With RMODE > 0 the kernel also runs the router gate for its tokens (the two
-// pre-expert stages are independent): for the team's i-th token, warp
-// i % TW of the team loads the token's logits before the norm passes and
-// selects its top-k after them (RMODE scores per lane, E <= 32 * RMODE).
-template <int TW, bool GC0, int RMODE>
+template <int TW, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     norm_quant_wide_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
     constexpr int P = TW * 32;
@@ -289,17 +277,8 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int sw = tid & 7;
     const int nblocks = H / 16;
 
-    int slot = 0, phase = 0, pbuf = 0, iter = 0;
-    constexpr int NL = RMODE > 0 ? RMODE : 4;
-    for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride, ++iter) {
-        // router: this warp's token?  issue its logit loads before the norm work
-        const bool router = RMODE > 0 && (iter % TW) == warp_in_team;
-        const bool route_valid = router && a.mask[t] != 0;
-        float lv[NL];
-        if constexpr (RMODE > 0) {
-            if (route_valid)
-                load_logits<NL>(a.logits + static_cast<size_t>(t) * a.E, a.E, lane, (a.E & 3) == 0, lv);
-        }
+    int slot = 0, phase = 0, pbuf = 0;
+    for (int t = blockIdx.x * NTEAM + team; t < M; t += team_stride) {
         const bool ok = mbar_wait_bounded(&tb[slot], phase, 4u);
         uint32_t wv[32];
         float b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -383,22 +362,6 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         *reinterpret_cast<uint4*>(prow + 16) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
         *reinterpret_cast<uint32_t*>(a.sf + static_cast<size_t>(t) * nblocks + 4 * tid) = sfw;
         }
-        if constexpr (RMODE > 0) {
-            if (router) {
-                int32_t* id_row = a.ids + static_cast<size_t>(t) * a.k;
-                float* w_row = a.weights + static_cast<size_t>(t) * a.k;
-                if (!route_valid) {
-                    if (lane < a.k) {
-                        id_row[lane] = -1;
-                        w_row[lane] = 0.0f;
-                    }
-                } else {
-                    uint32_t pick_key = 0u, pick_id = 0u;
-                    select_small<NL>(lv, a.bias, a.E, a.k, lane, (a.E & 3) == 0, pick_key, pick_id);
-                    route_write(a.logits + static_cast<size_t>(t) * a.E, a.k, lane, pick_id, id_row, w_row);
-                }
-            }
-        }
     }
     if (tid == 0)
         for (int f = cur->consumed; f < cur->issued; ++f)
@@ -450,7 +413,7 @@ cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a
     }
 }
 
-template <int TW, bool GC0, int RMODE>
+template <int TW, bool GC0>
 cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
     constexpr int P = TW * 32;
     constexpr int NTEAM = kConsumerThreads / P;
@@ -465,7 +428,7 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     NormQuantArgs a = args;
     a.nslot = nslot;
     const size_t smem = lay.total_bytes();
-    auto kern = norm_quant_wide_kernel<TW, GC0, RMODE>;
+    auto kern = norm_quant_wide_kernel<TW, GC0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -485,21 +448,19 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     return cudaLaunchKernelEx(&cfg, kern, tmap, a);
 }
 
-template <bool GC0, int RMODE>
+template <bool GC0>
 cudaError_t launch_nq_wide_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
     switch (TW) {
-        case 1: return launch_nq_wide<1, GC0, RMODE>(tmap, a, s);
-        case 2: return launch_nq_wide<2, GC0, RMODE>(tmap, a, s);
-        case 4: return launch_nq_wide<4, GC0, RMODE>(tmap, a, s);
-        case 8: return launch_nq_wide<8, GC0, RMODE>(tmap, a, s);
+        case 1: return launch_nq_wide<1, GC0>(tmap, a, s);
+        case 2: return launch_nq_wide<2, GC0>(tmap, a, s);
+        case 4: return launch_nq_wide<4, GC0>(tmap, a, s);
+        case 8: return launch_nq_wide<8, GC0>(tmap, a, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <int RMODE>
 cudaError_t launch_nq_wide_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
-    return a.gc == 0.0f ? launch_nq_wide_tw<true, RMODE>(TW, tmap, a, s)
-                        : launch_nq_wide_tw<false, RMODE>(TW, tmap, a, s);
+    return a.gc == 0.0f ? launch_nq_wide_tw<true>(TW, tmap, a, s) : launch_nq_wide_tw<false>(TW, tmap, a, s);
 }
 
 // gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
@@ -545,7 +506,7 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
     NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
     CUtensorMap tmap;
     int TW = 0;
-    if (wide_nq_plan(x, M, H, tp, tmap, TW)) return launch_nq_wide_gc<0>(TW, tmap, a, s);
+    if (wide_nq_plan(x, M, H, tp, tmap, TW)) return launch_nq_wide_gc(TW, tmap, a, s);
     const int hs = H / tp;
     const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
                      static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
@@ -560,17 +521,11 @@ cudaError_t launch_route_norm_quant(const float* logits, const float* bias, cons
                                     int32_t* ids, float* weights, const uint16_t* x, int M, int H, int tp,
                                     const uint16_t* w, float gc, float eps, const float* gs, uint8_t* packed,
                                     uint8_t* sf, cudaStream_t s) {
-    NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0, logits, bias, mask, E, k, ids, weights};
-    CUtensorMap tmap;
-    int TW = 0;
-    const int per_lane = (E + 31) / 32;
-    const int epl = (per_lane + 3) / 4 * 4;
-    if (epl <= 16 && wide_nq_plan(x, M, H, tp, tmap, TW)) {
-        if (epl <= 4) return launch_nq_wide_gc<4>(TW, tmap, a, s);
-        if (epl <= 8) return launch_nq_wide_gc<8>(TW, tmap, a, s);
-        return launch_nq_wide_gc<16>(TW, tmap, a, s);
-    }
-    // shapes the fused kernel does not take: the two kernels back to back
+    // The router is latency-bound and wants every warp slot of the SMs, the
+    // norm-quant is streaming-bound and holds their shared memory and most of
+    // their registers; run back to back (programmatic dependent launch
+    // overlaps their edges) they beat any single kernel that splits the SMs
+    // between the two.
     cudaError_t e = launch_route(logits, bias, mask, M, E, k, ids, weights, s);
     if (e != cudaSuccess) return e;
     return launch_norm_quant(x, M, H, tp, w, gc, eps, gs, packed, sf, s);

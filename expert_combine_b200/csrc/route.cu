@@ -147,6 +147,103 @@ __device__ __forceinline__ void select_small(const float (&lv)[EPL], const float
     }
 }
 
+// Two tokens at once (independent selection chains interleaved round by
+// round); tokens that are absent or masked are given all-zero keys and their
+// picks are ignored by the caller.
+template <int EPL>
+__device__ __forceinline__ void select_small2(const float (&la)[EPL], const float (&lb)[EPL], bool va, bool vb,
+                                              const float* bias, int E, int k, int lane, bool vec,
+                                              uint32_t& pick_a, uint32_t& pick_b) {
+    uint32_t ka[EPL], kb[EPL];
+#pragma unroll
+    for (int u = 0; u < EPL / 4; ++u) {
+        const int q = lane + 32 * u;
+        float4 b;
+        if (vec && 4 * q + 3 < E) {
+            b = __ldg(reinterpret_cast<const float4*>(bias) + q);
+        } else {
+            b.x = 4 * q + 0 < E ? __ldg(bias + 4 * q + 0) : 0.0f;
+            b.y = 4 * q + 1 < E ? __ldg(bias + 4 * q + 1) : 0.0f;
+            b.z = 4 * q + 2 < E ? __ldg(bias + 4 * q + 2) : 0.0f;
+            b.w = 4 * q + 3 < E ? __ldg(bias + 4 * q + 3) : 0.0f;
+        }
+        const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool in = 4 * q + i < E;
+            ka[4 * u + i] = (va && in) ? score_key(__fadd_rn(sigmoid_fixed(la[4 * u + i]), bb[i])) : 0u;
+            kb[4 * u + i] = (vb && in) ? score_key(__fadd_rn(sigmoid_fixed(lb[4 * u + i]), bb[i])) : 0u;
+        }
+    }
+    auto best_of = [&](const uint32_t (&key)[EPL], uint32_t& bk, int& bp) {
+        bk = 0u;
+        bp = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (key[i] > bk) {
+                bk = key[i];
+                bp = i;
+            }
+    };
+    uint32_t bka, bkb;
+    int bpa, bpb;
+    best_of(ka, bka, bpa);
+    best_of(kb, bkb, bpb);
+    for (int j = 0; j < k; ++j) {
+        const uint32_t ida = 4u * static_cast<uint32_t>(lane + 32 * (bpa >> 2)) + static_cast<uint32_t>(bpa & 3);
+        const uint32_t idb = 4u * static_cast<uint32_t>(lane + 32 * (bpb >> 2)) + static_cast<uint32_t>(bpb & 3);
+        const uint32_t ma = warp_max_u32(bka);
+        const uint32_t mb = warp_max_u32(bkb);
+        const uint32_t wa = warp_min_u32(bka == ma ? ida : 0xffffffffu);
+        const uint32_t wb = warp_min_u32(bkb == mb ? idb : 0xffffffffu);
+        if (bka == ma && ida == wa) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == bpa) ka[i] = 0u;
+            best_of(ka, bka, bpa);
+        }
+        if (bkb == mb && idb == wb) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i)
+                if (i == bpb) kb[i] = 0u;
+            best_of(kb, bkb, bpb);
+        }
+        if (lane == j) {
+            pick_a = wa;
+            pick_b = wb;
+        }
+    }
+}
+
+// Picks of two tokens written together (lane j < k holds pick j of each);
+// a token that is absent (t >= T) is skipped, a masked one gets -1 / 0.
+__device__ __forceinline__ void route_write2(const float* logits, int E, int k, int lane, int ta, int tb,
+                                             bool pa, bool pb, bool va, bool vb, uint32_t id_a, uint32_t id_b,
+                                             int32_t* ids, float* weights) {
+    const float* la = logits + static_cast<size_t>(ta) * E;
+    const float* lb = logits + static_cast<size_t>(tb) * E;
+    float sa = 0.0f, sb = 0.0f;
+    if (lane < k) {
+        if (va) sa = sigmoid_fixed(__ldg(la + id_a));
+        if (vb) sb = sigmoid_fixed(__ldg(lb + id_b));
+    }
+    float Sa = 0.0f, Sb = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        Sa = __fadd_rn(Sa, __shfl_sync(0xffffffffu, sa, j));
+        Sb = __fadd_rn(Sb, __shfl_sync(0xffffffffu, sb, j));
+    }
+    if (lane < k) {
+        if (pa) {
+            ids[static_cast<size_t>(ta) * k + lane] = va ? static_cast<int32_t>(id_a) : -1;
+            weights[static_cast<size_t>(ta) * k + lane] = va ? __fdiv_rn(sa, Sa) : 0.0f;
+        }
+        if (pb) {
+            ids[static_cast<size_t>(tb) * k + lane] = vb ? static_cast<int32_t>(id_b) : -1;
+            weights[static_cast<size_t>(tb) * k + lane] = vb ? __fdiv_rn(sb, Sb) : 0.0f;
+        }
+    }
+}
+
 // The picks' unbiased sigmoids, renormalised in pick order (lane j < k holds
 // pick j), written with the ids.
 __device__ __forceinline__ void route_write(const float* l, int k, int lane, uint32_t pick_id, int32_t* id_row,
@@ -246,6 +343,22 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
     const bool vec = (E & 3) == 0;
 
+    if constexpr (MODE > 0) {
+        // two tokens per iteration: t and t + nwarps
+        for (int t = warp; t < T; t += 2 * nwarps) {
+            const int tb = t + nwarps;
+            const bool pb = tb < T;
+            const bool va = mask[t] != 0;
+            const bool vb = pb && mask[tb] != 0;
+            float la[MODE], lb[MODE];
+            if (va) load_logits<MODE>(logits + static_cast<size_t>(t) * E, E, lane, vec, la);
+            if (vb) load_logits<MODE>(logits + static_cast<size_t>(tb) * E, E, lane, vec, lb);
+            uint32_t ida = 0u, idb = 0u;
+            select_small2<MODE>(la, lb, va, vb, bias, E, k, lane, vec, ida, idb);
+            route_write2(logits, E, k, lane, t, pb ? tb : t, true, pb, va, vb, ida, idb, ids, weights);
+        }
+        return;
+    }
     for (int t = warp; t < T; t += nwarps) {
         int32_t* id_row = ids + static_cast<size_t>(t) * k;
         float* w_row = weights + static_cast<size_t>(t) * k;
@@ -273,7 +386,9 @@ cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* 
                          int k, int32_t* ids, float* weights, cudaStream_t s) {
     const int per_lane = (E + 31) / 32;
     const int warps_per_cta = 8;
-    int grid = (T + warps_per_cta - 1) / warps_per_cta;
+    const int epl0 = ((E + 31) / 32 + 3) / 4 * 4;
+    const int tokens_per_warp = epl0 <= 16 ? 2 : 1;   // the small path routes two tokens per warp
+    int grid = (T + warps_per_cta * tokens_per_warp - 1) / (warps_per_cta * tokens_per_warp);
     const int cap = device_info().sm_count * 8;
     if (grid > cap) grid = cap;
     cudaLaunchConfig_t cfg = {};

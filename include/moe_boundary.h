@@ -93,17 +93,13 @@ int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* no
 
 /*
  * moe_route_norm_quant -- moe_route and norm_quant_nvfp4 of the same M tokens
- * in one launch.
+ * in one call.
  *
  * Source: as moe_route and norm_quant_nvfp4.  The two pre-expert stages read
- * disjoint inputs and are independent; TensorRT-LLM PR 21356 ("Where they
- * plug in") runs the pre-expert norm on an auxiliary stream while the router
- * runs on the current one.  Here one kernel does both: the team that
- * normalises and quantises token t also routes it.  Arguments and results
- * are those of the two calls with T = M, bit for bit.  When the fused kernel
- * does not take the sizes (E > 512, H < 2048, H % 64 != 0, or a rank-block
- * shard not a multiple of 512) the two kernels run back to back on `stream`.
- * Supported: the union of both calls' rules.
+ * disjoint inputs and are independent (TensorRT-LLM PR 21356, "Where they
+ * plug in", runs the pre-expert norm beside the router).  Both kernels are
+ * enqueued on `stream`, the router first; results are those of the two calls
+ * with T = M, bit for bit.  Supported: both calls' rules.
  */
 int moe_route_norm_quant(const float* logits, const float* bias, const uint8_t* token_mask, int E, int k,
                          int32_t* topk_ids, float* topk_weights, const uint16_t* x, int M, int H, int tp,
