@@ -357,28 +357,22 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             select_small2<MODE>(la, lb, va, vb, bias, E, k, lane, vec, ida, idb);
             route_write2(logits, E, k, lane, t, pb ? tb : t, true, pb, va, vb, ida, idb, ids, weights);
         }
-        return;
-    }
-    for (int t = warp; t < T; t += nwarps) {
-        int32_t* id_row = ids + static_cast<size_t>(t) * k;
-        float* w_row = weights + static_cast<size_t>(t) * k;
-        if (mask[t] == 0) {
-            if (lane < k) {
-                id_row[lane] = -1;
-                w_row[lane] = 0.0f;
+    } else {
+        for (int t = warp; t < T; t += nwarps) {
+            int32_t* id_row = ids + static_cast<size_t>(t) * k;
+            float* w_row = weights + static_cast<size_t>(t) * k;
+            if (mask[t] == 0) {
+                if (lane < k) {
+                    id_row[lane] = -1;
+                    w_row[lane] = 0.0f;
+                }
+                continue;
             }
-            continue;
-        }
-        const float* l = logits + static_cast<size_t>(t) * E;
-        uint32_t pick_key = 0u, pick_id = 0u;
-        if constexpr (MODE > 0) {
-            float lv[MODE];
-            load_logits<MODE>(l, E, lane, vec, lv);
-            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
-        } else {
+            const float* l = logits + static_cast<size_t>(t) * E;
+            uint32_t pick_key = 0u, pick_id = 0u;
             route_token_list<-MODE>(l, bias, E, k, lane, vec, pick_key, pick_id);
+            route_write(l, k, lane, pick_id, id_row, w_row);
         }
-        route_write(l, k, lane, pick_id, id_row, w_row);
     }
 }
 
