@@ -13,6 +13,13 @@ single moe_route_norm_quant call).
 Prints ONE JSON line (rank 0).  `value` is tokens/s over all ranks (weak
 scaling: every rank runs its own batch of 8192 tokens).  The per-step inputs
 (1.2 GB) are larger than the 126 MB L2, so no flush runs between steps.
+
+Timing: the K steps run back to back between two CUDA events on the launching
+stream (barrier + synchronize on both sides, max over ranks); no event sits
+between the kernels of the region, since one would keep the next kernel from
+launching early.  The per-stage times (`stages_ms`, and the combine's launch
+duration in `roofline`) come from a second region right after it: each stage
+alone, K back-to-back launches between two events.
 """
 from __future__ import annotations
 
@@ -272,17 +279,24 @@ def run_ours(args, world, rank, local):
                                     case.gc, case.eps, case.gs, topk_ids=ids, topk_weights=w,
                                     packed=packed, sf=sf)
 
-    def step(ev=None):
-        # ev: 3 events bracketing the pre-expert stages and the combine
-        if ev is not None:
-            ev[0].record(stream)
-        pre_expert()
-        if ev is not None:
-            ev[1].record(stream)
+    def combine():
         eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                           case.eps, out=out)
-        if ev is not None:
-            ev[2].record(stream)
+
+    def step():
+        pre_expert()
+        combine()
+
+    def timed(fn, n):
+        # n back-to-back calls between two events on the launching stream; an
+        # event between kernels would stop the next kernel's early launch, so
+        # none is recorded inside the region
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
+            fn()
+        t1.record(stream)
+        return t0, t1
 
     for _ in range(args.warmup):
         step()
@@ -290,19 +304,22 @@ def run_ours(args, world, rank, local):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
         time.sleep(0.3)
         t_wall = time.perf_counter()
-        for i in range(args.steps):
-            step(evs[i])
+        e0, e1 = timed(step, args.steps)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     barrier(world)
-    step_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(2)]
+    step_ms = e0.elapsed_time(e1)
+    # each stage alone, back to back, for the per-kernel launch durations
+    pre_ev = timed(pre_expert, args.steps)
+    cmb_ev = timed(combine, args.steps)
+    torch.cuda.synchronize()
+    stage_ms = [pre_ev[0].elapsed_time(pre_ev[1]) / args.steps,
+                cmb_ev[0].elapsed_time(cmb_ev[1]) / args.steps]
     combine_ms = stage_ms[1]
     step_ms_max = max_over_ranks(step_ms, world)
     ms_per_step = step_ms_max / args.steps
@@ -354,7 +371,8 @@ def run_ours(args, world, rank, local):
                          "bytes_per_launch": cmb_bytes_net,
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},
-            "stages_ms": {"route_norm_quant": stage_ms[0], "combine": stage_ms[1]},
+            "stages_ms": {"route_norm_quant": stage_ms[0], "combine": stage_ms[1],
+                          "how": "each stage alone, K back-to-back launches between two events"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,
