@@ -66,6 +66,7 @@ def _load():
                 "oc_norm_quant": (None, [P, i32, i32, i32, P, f32, f32, f32, P, P, P]),
                 "oc_combine": (None, [P, i64, i32, P, P, i32, i32, P, f32, f32, P]),
                 "oc_join": (None, [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32]),
+                "oc_dispatch": (None, [P, i32, i32, i32, i32, P, P, P]),
                 "oc_bf16_rn_n": (None, [P, i64, P]),
                 "oc_e4m3_rn_sat_n": (None, [P, i64, P]),
                 "oc_e2m1_code_n": (None, [P, i64, P]),
@@ -252,3 +253,19 @@ def join(residual, branch, gain, alpha: float, beta: float, eps: float,
     _load().oc_join(_ptr(r), _ptr(branch), _ptr(gain), float(alpha), float(beta), float(eps),
                     _ptr(nw), float(next_gc), float(next_eps), _ptr(p), T, H)
     return r, p
+
+
+def dispatch(ids, e0: int, E: int):
+    """Expert-grouped rows of the routing entries (lmdeploy PR 4835 "MoE gate
+    v2", commit notes: per-expert histogram and scan; en2f = -1 where no row).
+
+    ``ids`` int32 [T, k] of global expert ids; experts [e0, e0 + E) are this
+    rank's.  Returns ``offsets`` [E + 1], ``row_idx`` [T, k] (en2f) and
+    ``row_token`` [T * k] (token of each row, -1 past the last row)."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    offsets = np.empty(E + 1, dtype=np.int32)
+    row_idx = np.empty((T, k), dtype=np.int32)
+    row_token = np.empty(T * k, dtype=np.int32)
+    _load().oc_dispatch(_ptr(ids), T, k, e0, E, _ptr(offsets), _ptr(row_idx), _ptr(row_token))
+    return offsets, row_idx, row_token

@@ -24,7 +24,10 @@
  *    E4M3 block scale from the global scale, E2M1 thresholds, sign bit,
  *    nibble packing, linear scale layout, the rank-block input layout.
  *  - "MoE gate v2" (lmdeploy PR 4835), commit notes: a required token mask;
- *    invalid tokens produce no routing entries; absent rows marked -1.
+ *    invalid tokens produce no routing entries; absent rows marked -1; the
+ *    gate's routing entries are grouped per expert by a histogram and a scan
+ *    (the dispatch step), and en2f, the map from a routing entry to its row,
+ *    is cleared to -1 where no row exists.
  *
  * Where the pages leave a step open the oracle takes one fixed reading
  * (listed in the repository's design notes): the sigmoid's exp is the
@@ -421,6 +424,52 @@ void oc_join(float* residual, const uint16_t* branch, const uint16_t* gain, floa
         }
         free(g);
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* Dispatch: expert-grouped row layout of the routing entries           */
+/* ------------------------------------------------------------------ */
+
+/* ids [T, k] int32 holds global expert ids (-1: no entry).  This rank owns
+ * experts [e0, e0 + E); entry (t, j) is valid iff e0 <= ids[t, j] < e0 + E,
+ * and its local expert is ids[t, j] - e0.  Rows are grouped by local expert
+ * in ascending order; within one expert the entries keep their flattened
+ * order t * k + j (a stable counting sort: histogram, exclusive scan, then
+ * one ordered pass).  Outputs:
+ *   offsets   [E + 1]  first row of each expert; offsets[E] = R, the number
+ *                      of valid entries
+ *   row_idx   [T, k]   the row of entry (t, j) (the pages' en2f), -1 when the
+ *                      entry is invalid
+ *   row_token [T * k]  the token of row r for r < R, -1 for R <= r < T * k. */
+void oc_dispatch(const int32_t* ids, int T, int k, int e0, int E, int32_t* offsets,
+                 int32_t* row_idx, int32_t* row_token) {
+    const int64_t n = (int64_t)T * k;
+    int64_t* count = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t e = (int64_t)ids[i] - e0;
+        if (e >= 0 && e < E) count[e] += 1;
+    }
+    int64_t run = 0;
+    for (int e = 0; e < E; ++e) {
+        offsets[e] = (int32_t)run;
+        run += count[e];
+    }
+    offsets[E] = (int32_t)run;
+    int64_t* next = (int64_t*)malloc(sizeof(int64_t) * ((size_t)E + 1));
+    for (int e = 0; e < E; ++e) next[e] = offsets[e];
+    for (int64_t r = 0; r < n; ++r) row_token[r] = -1;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t e = (int64_t)ids[i] - e0;
+        if (e >= 0 && e < E) {
+            int64_t r = next[e]++;
+            row_idx[i] = (int32_t)r;
+            row_token[r] = (int32_t)(i / k);
+        } else {
+            row_idx[i] = -1;
+        }
+    }
+    free(next);
+    free(count);
 }
 
 /* ------------------------------------------------------------------ */
