@@ -335,6 +335,8 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = measured_peaks()
     achieved_cmb = cmb_bytes_net / (combine_ms * 1e-3) / 1e9
 
+    disp = None if args.no_dispatch else run_dispatch(eb, ids, E, dev, reps=max(5, min(args.steps, 200)))
+
     # end to end through the same calls with host buffers (pinned), copies inside
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
                                            pre_expert, steps=max(2, min(args.steps, 5)))
@@ -375,6 +377,7 @@ def run_ours(args, world, rank, local):
                           "how": "each stage alone, K back-to-back launches between two events"},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "dispatch": disp,
             "gpu_launches": 3 * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
@@ -384,6 +387,43 @@ def run_ours(args, world, rank, local):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout")
     return result
+
+
+def run_dispatch(eb, ids, E, dev, reps):
+    """The dispatch step (expert-grouped rows of this step's routing ids),
+    timed apart from the step: `reps` calls captured in one CUDA graph and
+    replayed between two events, so the time is the kernels' and not the
+    Python binding's."""
+    T, k = ids.shape
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    tok = torch.empty(T * k, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(1, eb.dispatch_workspace_size(T, k, E)), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            eb.moe_dispatch(ids, E, 0, off, idx, tok, ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            eb.moe_dispatch(ids, E, 0, off, idx, tok, ws)
+    g.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / reps
+    n = T * k
+    kernels = 1 if eb.dispatch_workspace_size(T, k, E) == 0 else 3
+    del g
+    return {"us": us, "entries": n, "experts": E, "kernels": kernels,
+            "bytes": 12 * n, "gbs": 12 * n / (us * 1e-6) / 1e9,
+            "bound": "latency", "how": f"{reps} calls in one CUDA graph, replayed between two events",
+            "valid_rows": int(off[-1].item())}
 
 
 def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, pre_expert, steps):
@@ -428,6 +468,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default: the workload's 8192); smaller for profiling")
+    ap.add_argument("--no-dispatch", action="store_true",
+                    help="skip the separate timing of the dispatch step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--joint", action="store_true",
                     help="enqueue the pre-expert stages with the joint moe_route_norm_quant call")

@@ -1,4 +1,5 @@
-"""B200-native per-token MoE boundary: router gate, RMSNorm + NVFP4, expert combine, residual join.
+"""B200-native per-token MoE boundary: router gate, RMSNorm + NVFP4, dispatch, expert combine,
+residual join.
 
 Thin Python binding over the C ABI of ``libmoe_boundary.so`` (declared in
 ``include/moe_boundary.h``).  This package only marshals arguments: it checks
@@ -13,16 +14,19 @@ from ._lib import (  # noqa: F401
     MoEBoundaryError,
     STAGE_COMBINE,
     STAGE_COMBINE_JOIN,
+    STAGE_DISPATCH,
     STAGE_JOIN,
     STAGE_NORM_QUANT,
     STAGE_ROUTE,
     STAGE_ROUTE_NORM_QUANT,
     device_status,
+    dispatch_workspace_size,
     expert_combine,
     expert_combine_join,
     last_error,
     lib_path,
     load,
+    moe_dispatch,
     moe_route,
     moe_route_norm_quant,
     norm_quant_nvfp4,

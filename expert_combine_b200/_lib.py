@@ -16,6 +16,7 @@ STAGE_COMBINE = 2
 STAGE_JOIN = 3
 STAGE_COMBINE_JOIN = 4
 STAGE_ROUTE_NORM_QUANT = 5
+STAGE_DISPATCH = 6
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +61,7 @@ def load() -> ctypes.CDLL:
                                         f32, P, f32, f32, P, P],
                 "moe_route_norm_quant": [P, P, P, i32, i32, P, P, P, i32, i32, i32, P, f32, f32, P, P,
                                          P, P],
+                "moe_dispatch": [P, i32, i32, i32, i32, P, P, P, P, ctypes.c_size_t, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
                 "mb_last_error": [],
                 "mb_device_status": [],
@@ -68,6 +70,8 @@ def load() -> ctypes.CDLL:
                 fn = getattr(lib, name)
                 fn.argtypes = args
                 fn.restype = ctypes.c_char_p if name == "mb_last_error" else ctypes.c_int
+            lib.moe_dispatch_workspace_size.argtypes = [i32, i32, i32]
+            lib.moe_dispatch_workspace_size.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -282,3 +286,45 @@ def expert_combine_join(expert_out: torch.Tensor, num_rows: int, row_idx: torch.
                                       float(next_gc), float(next_eps), _ptr(next_prenorm),
                                       _stream(stream)))
     return out, next_prenorm
+
+
+def dispatch_workspace_size(T: int, k: int, E: int) -> int:
+    """Bytes of device workspace moe_dispatch needs for T tokens x k picks over E experts."""
+    return int(load().moe_dispatch_workspace_size(T, k, E))
+
+
+def moe_dispatch(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0,
+                 expert_offsets: Optional[torch.Tensor] = None, row_idx: Optional[torch.Tensor] = None,
+                 row_token: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None):
+    """Expert-grouped rows of the routing entries ->
+    (expert_offsets int32 [E + 1], row_idx int32 [T, k], row_token int32 [T * k]).
+
+    ``workspace`` is a uint8 CUDA tensor of at least ``dispatch_workspace_size``
+    bytes; when omitted, one is allocated here (the library itself never
+    allocates)."""
+    _want(topk_ids, torch.int32, "topk_ids")
+    T, k = topk_ids.shape
+    E = int(num_experts)
+    dev = topk_ids.device
+    if expert_offsets is None:
+        expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_idx is None:
+        row_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _want(expert_offsets, torch.int32, "expert_offsets")
+    _want(row_idx, torch.int32, "row_idx")
+    _want(row_token, torch.int32, "row_token")
+    if expert_offsets.numel() != E + 1 or row_idx.shape != (T, k) or row_token.numel() != T * k:
+        raise ValueError("moe_dispatch: shape mismatch")
+    need = dispatch_workspace_size(T, k, E)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _want(workspace, torch.uint8, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _check("moe_dispatch", load().moe_dispatch(_ptr(topk_ids), T, k, int(expert_begin), E,
+                                               _ptr(expert_offsets), _ptr(row_idx), _ptr(row_token),
+                                               _ptr(workspace), ws_bytes, _stream(stream)))
+    return expert_offsets, row_idx, row_token

@@ -1,5 +1,6 @@
 // api.cu -- the C ABI (include/moe_boundary.h): argument checks, status codes
 // and launches.  No allocation, no synchronisation, no host fallback.
+#include <climits>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -71,6 +72,11 @@ int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp) {
             return (hidden_ok(H) && k >= 1 && k <= kMaxTopK) ? 1 : 0;
         case MB_STAGE_JOIN:
             return hidden_ok(H) ? 1 : 0;
+        case MB_STAGE_DISPATCH:
+            return (k >= 1 && k <= kMaxTopK && E >= 1 && E <= kMaxExperts &&
+                    static_cast<int64_t>(T) * k <= INT32_MAX)
+                       ? 1
+                       : 0;
         case MB_STAGE_ROUTE_NORM_QUANT:
             return (moe_boundary_supported(MB_STAGE_ROUTE, T, H, E, k, tp) &&
                     moe_boundary_supported(MB_STAGE_NORM_QUANT, T, H, E, k, tp))
@@ -216,6 +222,36 @@ int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, con
     return cuda_status(launch_combine(expert_out, num_rows, H, row_idx, weights, T, k, norm_w, gain_center,
                                       eps, out, j, static_cast<cudaStream_t>(stream)),
                        "expert_combine_join");
+}
+
+size_t moe_dispatch_workspace_size(int T, int k, int E) {
+    if (T < 0 || k < 1 || E < 1) return 0;
+    return dispatch_workspace_bytes(static_cast<int64_t>(T) * k, E);
+}
+
+int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
+                 int32_t* row_idx, int32_t* row_token, void* workspace, size_t workspace_bytes, void* stream) {
+    const char* fn = "moe_dispatch";
+    if (T < 0 || k < 0 || E < 0 || expert_begin < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative argument", fn);
+    if (static_cast<int64_t>(expert_begin) + E > INT32_MAX)
+        return fail(MB_ERR_INVALID_ARG, "%s: expert_begin + E overflows int32", fn);
+    if (!moe_boundary_supported(MB_STAGE_DISPATCH, T, 0, E, k, 1))
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs 1 <= k <= %d, 1 <= E <= %d and T * k < 2^31 (T=%d, k=%d, E=%d)",
+                    fn, kMaxTopK, kMaxExperts, T, k, E);
+    if (!expert_offsets || (T > 0 && (!topk_ids || !row_idx || !row_token)))
+        return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(expert_offsets) || !aligned16(topk_ids) || !aligned16(row_idx) || !aligned16(row_token))
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    const size_t need = dispatch_workspace_bytes(static_cast<int64_t>(T) * k, E);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(MB_ERR_INVALID_ARG, "%s: needs a workspace of %zu bytes (got %zu)", fn, need,
+                        workspace ? workspace_bytes : static_cast<size_t>(0));
+        if (!aligned16(workspace)) return fail(MB_ERR_INVALID_ARG, "%s: workspace must be 16-byte aligned", fn);
+    }
+    return cuda_status(launch_dispatch(topk_ids, T, k, expert_begin, E, expert_offsets, row_idx, row_token,
+                                       workspace, static_cast<cudaStream_t>(stream)),
+                       fn);
 }
 
 int mb_device_status(void) {

@@ -41,6 +41,12 @@ cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const i
 cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,
                                  cudaStream_t s);
 
+// Dispatch: workspace bytes for n = T * k entries (0 when one tile holds
+// them all), and the launch (one kernel, or three with the workspace).
+size_t dispatch_workspace_bytes(int64_t n, int E);
+cudaError_t launch_dispatch(const int32_t* ids, int T, int k, int e0, int E, int32_t* offsets, int32_t* row_idx,
+                            int32_t* row_token, void* workspace, cudaStream_t s);
+
 // Largest H the row kernels take (16-element blocks, at most 1024 per row).
 constexpr int kMaxHidden = 16384;
 constexpr int kMaxTopK = 32;

@@ -6,3 +6,4 @@
 #include "combine.cu"
 #include "route.cu"
 #include "norm_quant.cu"
+#include "dispatch.cu"

@@ -219,6 +219,35 @@ def make_case(name: str, device="cpu", seed: Optional[int] = None, T: Optional[i
     return case
 
 
+def make_topk_ids(T: int, k: int, E: int, seed: int, masked_frac: float = 0.05,
+                  invalid_frac: float = 0.0, expert_begin: int = 0, span: Optional[int] = None,
+                  distinct: bool = True, device="cpu") -> torch.Tensor:
+    """Router-shaped expert ids [T, k] int32 (dispatch input), seeded.
+
+    Each token draws k experts from [expert_begin, expert_begin + span)
+    (span defaults to E), distinct within the token unless ``distinct`` is
+    False; ``masked_frac`` of the tokens are masked (all -1) and
+    ``invalid_frac`` of the remaining slots are set to -1."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    span = E if span is None else span
+    ids = torch.empty(T, k, dtype=torch.int64)
+    step = max(1, (1 << 24) // max(span, 1))
+    for s in range(0, T, step):
+        e = min(T, s + step)
+        if distinct:
+            keys = torch.rand(e - s, span, generator=gen)
+            ids[s:e] = keys.topk(k, dim=1).indices
+        else:
+            ids[s:e] = torch.randint(0, span, (e - s, k), generator=gen)
+    ids += expert_begin
+    masked = torch.rand(T, generator=gen) < masked_frac
+    ids[masked] = -1
+    if invalid_frac > 0:
+        ids[torch.rand(T, k, generator=gen) < invalid_frac] = -1
+    return ids.to(torch.int32).to(device)
+
+
 def as_u16(t: torch.Tensor):
     """BF16 tensor -> numpy uint16 array of its bits (host copy)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")

@@ -25,6 +25,7 @@
 #ifndef MOE_BOUNDARY_H
 #define MOE_BOUNDARY_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -175,6 +176,44 @@ int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, con
                         const uint16_t* next_w, float next_gc, float next_eps,
                         uint16_t* next_prenorm, void* stream);
 
+/*
+ * moe_dispatch -- expert-grouped rows of the routing entries: the dispatch
+ * step between the router (moe_route) and the experts, producing the
+ * row_idx that expert_combine reads.
+ *
+ * Source: lmdeploy PR 4835 "MoE gate v2", commit notes (the routing entries
+ * are grouped per expert by a histogram and an exclusive scan, hierarchical
+ * over CTAs for large expert counts; tokens without routing entries get no
+ * rows; en2f, the row of each routing entry, is cleared to -1 where no row
+ * exists; the routed count is passed on).
+ *
+ * Entry i = t * k + j of topk_ids is valid iff expert_begin <= topk_ids[i] <
+ * expert_begin + E (the experts of this rank; -1, the router's mark for a
+ * masked token, is never valid); its local expert is e = topk_ids[i] -
+ * expert_begin.  Rows are grouped by e ascending; inside one expert the
+ * entries keep the order of i (a stable counting sort), so tokens ascend.
+ *
+ *   topk_ids        [T, k] int32 (global expert ids)
+ *   expert_offsets  [E + 1] int32 (out): first row of each expert;
+ *                   expert_offsets[E] = R, the number of valid entries
+ *   row_idx         [T, k] int32 (out): the row of entry i (en2f), -1 when
+ *                   the entry is invalid
+ *   row_token       [T * k] int32 (out): the token of row r for r < R, -1 for
+ *                   R <= r < T * k
+ *   workspace       device scratch of moe_dispatch_workspace_size(T, k, E)
+ *                   bytes, 16-byte aligned, owned by the caller; may be NULL
+ *                   when that size is 0 (T * k <= 4096).  Its contents need
+ *                   no initialisation and are not kept between calls, but
+ *                   two calls that overlap on the GPU need two workspaces.
+ * Returns MB_ERR_INVALID_ARG when the workspace is missing or too small.
+ * T == 0 still writes expert_offsets (all zero); the other pointers may then
+ * be NULL.  Integer only: the result does not depend on the launch shape.
+ * Supported: 1 <= k <= 32, 1 <= E <= 4096, T * k < 2^31, expert_begin >= 0.
+ */
+size_t moe_dispatch_workspace_size(int T, int k, int E);
+int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
+                 int32_t* row_idx, int32_t* row_token, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Stage ids for moe_boundary_supported(). */
 enum {
     MB_STAGE_ROUTE = 0,
@@ -183,6 +222,7 @@ enum {
     MB_STAGE_JOIN = 3,
     MB_STAGE_COMBINE_JOIN = 4,
     MB_STAGE_ROUTE_NORM_QUANT = 5,
+    MB_STAGE_DISPATCH = 6,
 };
 
 /*

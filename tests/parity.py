@@ -99,6 +99,14 @@ def oracle_combine(case: synth.Case, wt_host, tokens=None):
                           case.post_gc, case.eps)
 
 
+def check_combine_rows(got_u16, rows_u16, R, row_idx, wt, post_w_u16, gc, eps):
+    """A combine output against the oracle's combine of the same rows."""
+    want = oracle.combine(rows_u16, R, row_idx, wt, post_w_u16, gc, eps)
+    d = bf16_ulp_diff(got_u16, want)
+    assert d.max() <= 1, f"combine differs by {d.max()} BF16 ulp at {np.argwhere(d > 1)[:5]}"
+    return int((d > 0).sum())
+
+
 def check_combine(case: synth.Case, tokens=None, wt=None, wt_host=None):
     if wt is None:
         wt = case.comb_wt

@@ -21,8 +21,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for fn in ("moe_route", "norm_quant_nvfp4", "expert_combine", "residual_join",
-               "expert_combine_join", "moe_boundary_supported", "mb_last_error",
-               "mb_device_status"):
+               "expert_combine_join", "moe_dispatch", "moe_dispatch_workspace_size",
+               "moe_boundary_supported", "mb_last_error", "mb_device_status"):
         assert fn in names
 
 
@@ -44,6 +44,11 @@ def test_supported_predicate():
     assert eb.supported(eb.STAGE_COMBINE, 8, 8192, 0, 8)
     assert not eb.supported(eb.STAGE_COMBINE, 8, 8200, 0, 8)
     assert eb.supported(eb.STAGE_JOIN, 8, 16384)
+    assert eb.supported(eb.STAGE_DISPATCH, 8192, 0, 256, 8)
+    assert eb.supported(eb.STAGE_DISPATCH, 65536, 0, 4096, 32)
+    assert not eb.supported(eb.STAGE_DISPATCH, 8, 0, 0, 8)
+    assert not eb.supported(eb.STAGE_DISPATCH, 8, 0, 4097, 8)
+    assert not eb.supported(eb.STAGE_DISPATCH, 1 << 27, 0, 256, 32)
     assert not eb.supported(99, 8, 16)
 
 
@@ -68,6 +73,28 @@ def test_bad_arguments_are_rejected_before_any_launch():
     a = ctypes.c_void_p(0x1000)
     assert lib.residual_join(a, a, a, 1.0, 0.5, 1e-6, a, 1.0, 1e-6, N, 4, 64, N) == 1
     assert "both" in eb.last_error()
+    # dispatch: sizes, pointers and the workspace are checked before any launch
+    Z = ctypes.c_size_t(0)
+    assert lib.moe_dispatch(N, 4, 8, 0, 0, N, N, N, N, Z, N) == 2
+    assert lib.moe_dispatch(N, 4, 8, -1, 256, N, N, N, N, Z, N) == 1
+    assert lib.moe_dispatch(N, 4, 8, 0, 256, N, N, N, N, Z, N) == 1
+    assert "null" in eb.last_error()
+    assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, N, Z, N) == 1
+    assert "workspace" in eb.last_error()
+    need = eb.dispatch_workspace_size(8192, 8, 256)
+    assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, a, ctypes.c_size_t(need - 1), N) == 1
+    assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, odd, ctypes.c_size_t(need), N) == 1
+    assert "aligned" in eb.last_error()
+
+
+def test_dispatch_workspace_size():
+    # one tile (<= 4096 entries) needs none; beyond, one count per tile and
+    # expert plus the totals
+    assert eb.dispatch_workspace_size(512, 8, 256) == 0
+    assert eb.dispatch_workspace_size(0, 8, 256) == 0
+    assert eb.dispatch_workspace_size(513, 8, 256) == (2 + 1) * 256 * 4
+    assert eb.dispatch_workspace_size(8192, 8, 256) == (16 + 1) * 256 * 4
+    assert eb.dispatch_workspace_size(65536, 22, 512) == (352 + 1) * 512 * 4
 
 
 def test_binding_refuses_cpu_tensors():
