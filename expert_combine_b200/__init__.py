@@ -27,6 +27,7 @@ from ._lib import (  # noqa: F401
     lib_path,
     load,
     moe_dispatch,
+    moe_dispatch_noalloc,
     moe_route,
     moe_route_norm_quant,
     norm_quant_nvfp4,

@@ -62,6 +62,7 @@ def load() -> ctypes.CDLL:
                 "moe_route_norm_quant": [P, P, P, i32, i32, P, P, P, i32, i32, i32, P, f32, f32, P, P,
                                          P, P],
                 "moe_dispatch": [P, i32, i32, i32, i32, P, P, P, P, ctypes.c_size_t, P],
+                "moe_dispatch_noalloc": [P, i32, i32, i32, i32, P, P, P, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
                 "mb_last_error": [],
                 "mb_device_status": [],
@@ -327,4 +328,35 @@ def moe_dispatch(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0
     _check("moe_dispatch", load().moe_dispatch(_ptr(topk_ids), T, k, int(expert_begin), E,
                                                _ptr(expert_offsets), _ptr(row_idx), _ptr(row_token),
                                                _ptr(workspace), ws_bytes, _stream(stream)))
+    return expert_offsets, row_idx, row_token
+
+
+def moe_dispatch_noalloc(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0,
+                         expert_offsets: Optional[torch.Tensor] = None,
+                         row_idx: Optional[torch.Tensor] = None,
+                         row_token: Optional[torch.Tensor] = None, stream=None):
+    """moe_dispatch with the library's fixed scratch array instead of a workspace,
+    for callers that cannot allocate device memory on the calling path.
+
+    Pass preallocated outputs to allocate nothing at all (outputs left as None
+    are allocated here).  Calls that overlap on the GPU share the scratch and
+    race; see the C header for the size limit."""
+    _want(topk_ids, torch.int32, "topk_ids")
+    T, k = topk_ids.shape
+    E = int(num_experts)
+    dev = topk_ids.device
+    if expert_offsets is None:
+        expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_idx is None:
+        row_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _want(expert_offsets, torch.int32, "expert_offsets")
+    _want(row_idx, torch.int32, "row_idx")
+    _want(row_token, torch.int32, "row_token")
+    if expert_offsets.numel() != E + 1 or row_idx.shape != (T, k) or row_token.numel() != T * k:
+        raise ValueError("moe_dispatch_noalloc: shape mismatch")
+    _check("moe_dispatch_noalloc",
+           load().moe_dispatch_noalloc(_ptr(topk_ids), T, k, int(expert_begin), E, _ptr(expert_offsets),
+                                       _ptr(row_idx), _ptr(row_token), _stream(stream)))
     return expert_offsets, row_idx, row_token

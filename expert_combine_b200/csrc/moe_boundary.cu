@@ -7,3 +7,4 @@
 #include "route.cu"
 #include "norm_quant.cu"
 #include "dispatch.cu"
+#include "dispatch_noalloc.cu"

@@ -214,6 +214,33 @@ size_t moe_dispatch_workspace_size(int T, int k, int E);
 int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
                  int32_t* row_idx, int32_t* row_token, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * moe_dispatch_noalloc -- moe_dispatch without a caller workspace, for
+ * callers that cannot allocate device memory.
+ *
+ * No counterpart on the reference pages: this entry point exists for callers
+ * that have no device memory to hand over -- their memory belongs to an
+ * allocator they cannot reach from this call site, or they must not call
+ * cudaMalloc/cudaFree on the hot path (those calls can synchronise the whole
+ * device), or the GPU's memory is already spoken for.  The call allocates
+ * nothing: its scratch is a fixed 1 MiB array compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ * Arguments, outputs and results are those of moe_dispatch (bit for bit).
+ * Limit: the inputs must fit the array, (ceil(T * k / 4096) + 1) * E * 4 <=
+ * 1 MiB (for example T * k up to about 4.19 M entries at E = 256, 413 K at
+ * E = 2560); larger calls return MB_ERR_UNSUPPORTED without launching.
+ * Every call on a device shares the one array: two calls whose kernels
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * it and can return wrong rows.  Nothing in the array needs to start at zero
+ * (each call writes every count it reads), and it keeps the last call's
+ * counts.  The first call on a device looks up the array's device address
+ * (synchronous, once per device, with that device current); make that first
+ * call before any stream capture begins.
+ */
+int moe_dispatch_noalloc(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
+                         int32_t* row_idx, int32_t* row_token, void* stream);
+
 /* Stage ids for moe_boundary_supported(). */
 enum {
     MB_STAGE_ROUTE = 0,
