@@ -686,6 +686,7 @@ int team_warps(int H);   // norm_quant.cu
 cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const int32_t* row_idx,
                            const float* wt, int T, int k, const uint16_t* w, float gc, float eps,
                            uint16_t* out, const JoinArgs& join, cudaStream_t s) {
+    if (cluster_path(T, H)) return launch_combine_cluster(expert_out, R, H, row_idx, wt, T, k, w, gc, eps, out, join, s);
     const CombineArgs a{expert_out, R, H, row_idx, wt, T, k, w, gc, eps, out, join, 0};
     const int TW = team_warps(H);
     const bool fused = join.residual != nullptr;
@@ -706,6 +707,7 @@ cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const i
 
 cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,
                                  cudaStream_t s) {
+    if (cluster_path(T, H)) return launch_join_cluster(branch, T, H, join, s);
     switch (team_warps(H)) {
         case 1: return launch_rj<1>(branch, T, H, join, s);
         case 2: return launch_rj<2>(branch, T, H, join, s);

@@ -41,6 +41,17 @@ cudaError_t launch_combine(const uint16_t* expert_out, int64_t R, int H, const i
 cudaError_t launch_residual_join(const uint16_t* branch, int T, int H, const JoinArgs& join,
                                  cudaStream_t s);
 
+// Few tokens (decode): combine / join with one token per thread-block cluster
+// (decode.cu) while T * next_pow2(H / 16) <= SMs * kClusterThreadsPerSM (148
+// tokens at H = 8192 on B200); the row kernels take larger T.  Bit-identical
+// results.
+constexpr int kClusterThreadsPerSM = 512;
+bool cluster_path(int T, int H);
+cudaError_t launch_combine_cluster(const uint16_t* expert_out, int64_t R, int H, const int32_t* row_idx,
+                                   const float* wt, int T, int k, const uint16_t* w, float gc, float eps,
+                                   uint16_t* out, const JoinArgs& join, cudaStream_t s);
+cudaError_t launch_join_cluster(const uint16_t* branch, int T, int H, const JoinArgs& join, cudaStream_t s);
+
 // Dispatch: workspace bytes for n = T * k entries (0 when one tile holds
 // them all), and the launch (one kernel, or three with the workspace).
 size_t dispatch_workspace_bytes(int64_t n, int E);

@@ -6,5 +6,6 @@
 #include "combine.cu"
 #include "route.cu"
 #include "norm_quant.cu"
+#include "decode.cu"
 #include "dispatch.cu"
 #include "dispatch_noalloc.cu"
