@@ -336,6 +336,7 @@ def run_ours(args, world, rank, local):
     achieved_cmb = cmb_bytes_net / (combine_ms * 1e-3) / 1e9
 
     disp = None if args.no_dispatch else run_dispatch(eb, ids, E, dev, reps=max(5, min(args.steps, 200)))
+    dec = None if args.no_decode else run_decode(eb, dev, reps=max(5, min(args.steps, 100)))
 
     # end to end through the same calls with host buffers (pinned), copies inside
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
@@ -378,6 +379,7 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "dispatch": disp,
+            "decode": dec,
             "gpu_launches": 3 * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
@@ -391,24 +393,35 @@ def run_ours(args, world, rank, local):
 
 def run_dispatch(eb, ids, E, dev, reps):
     """The dispatch step (expert-grouped rows of this step's routing ids),
-    timed apart from the step: `reps` calls captured in one CUDA graph and
-    replayed between two events, so the time is the kernels' and not the
-    Python binding's."""
+    timed apart from the step in CUDA-graph replays, so the time is the
+    kernels' and not the Python binding's."""
     T, k = ids.shape
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
     idx = torch.empty(T, k, dtype=torch.int32, device=dev)
     tok = torch.empty(T * k, dtype=torch.int32, device=dev)
     ws = torch.empty(max(1, eb.dispatch_workspace_size(T, k, E)), dtype=torch.uint8, device=dev)
+    us = _graph_us(lambda: eb.moe_dispatch(ids, E, 0, off, idx, tok, ws), reps, dev)
+    n = T * k
+    kernels = 1 if eb.dispatch_workspace_size(T, k, E) == 0 else 3
+    return {"us": us, "entries": n, "experts": E, "kernels": kernels,
+            "bytes": 12 * n, "gbs": 12 * n / (us * 1e-6) / 1e9,
+            "bound": "latency", "how": f"{reps} calls per CUDA graph, one replay between two events",
+            "valid_rows": int(off[-1].item())}
+
+
+def _graph_us(fn, reps, dev):
+    """Microseconds per call of `fn`: `reps` calls captured in one CUDA graph,
+    replayed once between two events (launch-latency-sized work)."""
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(side):
         for _ in range(3):
-            eb.moe_dispatch(ids, E, 0, off, idx, tok, ws)
+            fn()
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for _ in range(reps):
-            eb.moe_dispatch(ids, E, 0, off, idx, tok, ws)
+            fn()
     g.replay()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -416,14 +429,47 @@ def run_dispatch(eb, ids, E, dev, reps):
     g.replay()
     t1.record()
     torch.cuda.synchronize()
-    us = t0.elapsed_time(t1) * 1e3 / reps
-    n = T * k
-    kernels = 1 if eb.dispatch_workspace_size(T, k, E) == 0 else 3
     del g
-    return {"us": us, "entries": n, "experts": E, "kernels": kernels,
-            "bytes": 12 * n, "gbs": 12 * n / (us * 1e-6) / 1e9,
-            "bound": "latency", "how": f"{reps} calls in one CUDA graph, replayed between two events",
-            "valid_rows": int(off[-1].item())}
+    return t0.elapsed_time(t1) * 1e3 / reps
+
+
+def run_decode(eb, dev, reps):
+    """The decode workload (128 tokens, H=8192, E=256, k=8, the gated residual
+    join and next prenorm fused into the combine): latency of each stage and
+    of the whole boundary, from CUDA-graph replays."""
+    from expert_combine_b200 import synth
+    case = synth.make_case("decode", device=dev, seed=synth.SEEDS["decode"])
+    T, H, k = case.T, case.H, case.k
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    packed = torch.empty(T, H // 2, dtype=torch.uint8, device=dev)
+    sf = torch.empty(T, H // 16, dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    nxt = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    res = case.residual.clone()
+
+    def route():
+        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+
+    def nq():
+        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed, sf=sf)
+
+    def cj():
+        eb.expert_combine_join(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
+                               case.eps, res, case.gain, case.alpha, case.beta, case.eps, case.next_w,
+                               case.next_gc, case.eps, out=out, next_prenorm=nxt)
+
+    def step():
+        route()
+        nq()
+        cj()
+
+    r = {"workload": f"decode T={T} H={H} E={case.E} k={k}, join + next prenorm fused",
+         "route_us": _graph_us(route, reps, dev), "norm_quant_us": _graph_us(nq, reps, dev),
+         "combine_join_us": _graph_us(cj, reps, dev), "step_us": _graph_us(step, reps, dev),
+         "how": f"{reps} calls per CUDA graph, one replay between two events"}
+    r["tokens_per_s"] = T / (r["step_us"] * 1e-6)
+    return r
 
 
 def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, pre_expert, steps):
@@ -468,6 +514,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default: the workload's 8192); smaller for profiling")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the separate latency of the decode-sized boundary")
     ap.add_argument("--no-dispatch", action="store_true",
                     help="skip the separate timing of the dispatch step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
