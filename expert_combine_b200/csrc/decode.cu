@@ -48,6 +48,13 @@ __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Final barrier: only keeps every CTA's shared memory alive until all remote
+// reads of it are done (their values were consumed before this point), so no
+// memory ordering is needed and pending global stores are not waited for.
+__device__ __forceinline__ void cluster_exit_sync() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
 // The float at `local` (a shared-memory address of this CTA) in the CTA of
 // cluster rank `rank`.
 __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
@@ -226,7 +233,8 @@ __global__ void __launch_bounds__(TPB) boundary_cluster_kernel(const DecodeArgs 
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) bw[i] = pack_bf16x2_rn(acc[i]);
-        if (a.out != nullptr && has) store_block16(a.out + static_cast<size_t>(t) * H + col, bw);
+        if constexpr (!JOIN)
+            if (a.out != nullptr && has) store_block16(a.out + static_cast<size_t>(t) * H + col, bw);
     } else {
         if (has) load_block16(a.branch + static_cast<size_t>(t) * H + col, bw);
         else
@@ -236,20 +244,20 @@ __global__ void __launch_bounds__(TPB) boundary_cluster_kernel(const DecodeArgs 
 
     if constexpr (JOIN) {
         const JoinArgs& jn = a.join;
-        // g = bf16(gain * branch), n = bf16(g * inv(g)), r' = alpha r + beta n
-        uint32_t gw[8], gg[8];
-        if (has) load_block16(jn.gain + col, gw);
-        else
-#pragma unroll
-            for (int i = 0; i < 8; ++i) gw[i] = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) gg[i] = pack_bf16x2_rn(mul2(unpack_bf16x2(gw[i]), unpack_bf16x2(bw[i])));
-        const float inv_g = inv_rms_h(row_sum<NW, C>(block_sumsq_bf16(gg), wg, cg), fH, rH, pow2, jn.eps);
-        const float2 inv_g2 = make_float2(inv_g, inv_g);
-        const float2 alpha2 = make_float2(jn.alpha, jn.alpha);
-        const float2 beta2 = make_float2(jn.beta, jn.beta);
-        float* rrow = jn.residual + static_cast<size_t>(t) * H + col;
+        // g = bf16(gain * branch), n = bf16(g * inv(g)), r' = alpha r + beta n; every
+        // global store waits until the last cluster reduction is done
+        uint32_t gw[8], nw2[8];
         float2 r[8];
+        const bool hn = has && jn.next_w != nullptr;
+        const float* rrow = jn.residual + static_cast<size_t>(t) * H + col;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint4 g4 = make_uint4(0u, 0u, 0u, 0u), n4 = make_uint4(0u, 0u, 0u, 0u);
+            if (has) g4 = *reinterpret_cast<const uint4*>(jn.gain + col + 8 * c);
+            if (hn) n4 = *reinterpret_cast<const uint4*>(jn.next_w + col + 8 * c);
+            gw[4 * c] = g4.x; gw[4 * c + 1] = g4.y; gw[4 * c + 2] = g4.z; gw[4 * c + 3] = g4.w;
+            nw2[4 * c] = n4.x; nw2[4 * c + 1] = n4.y; nw2[4 * c + 2] = n4.z; nw2[4 * c + 3] = n4.w;
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -257,33 +265,39 @@ __global__ void __launch_bounds__(TPB) boundary_cluster_kernel(const DecodeArgs 
             r[2 * c] = make_float2(v.x, v.y);
             r[2 * c + 1] = make_float2(v.z, v.w);
         }
+        uint32_t gg[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gg[i] = pack_bf16x2_rn(mul2(unpack_bf16x2(gw[i]), unpack_bf16x2(bw[i])));
+        const float inv_g = inv_rms_h(row_sum<NW, C>(block_sumsq_bf16(gg), wg, cg), fH, rH, pow2, jn.eps);
+        const float2 inv_g2 = make_float2(inv_g, inv_g);
+        const float2 alpha2 = make_float2(jn.alpha, jn.alpha);
+        const float2 beta2 = make_float2(jn.beta, jn.beta);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float2 n = unpack_bf16x2(pack_bf16x2_rn(mul2(unpack_bf16x2(gg[i]), inv_g2)));
             r[i] = add2(mul2(alpha2, r[i]), mul2(beta2, n));
         }
-        if (has)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<float4*>(rrow + 4 * c) =
-                    make_float4(r[2 * c].x, r[2 * c].y, r[2 * c + 1].x, r[2 * c + 1].y);
+        uint32_t pw[8];
         if (jn.next_w != nullptr) {
             // p = bf16((r' * (next_gc + next_w)) * inv(r'))
             const float inv_r = inv_rms_h(row_sum<NW, C>(block_sumsq_f32(r), wr, cr), fH, rH, pow2, jn.next_eps);
             const float2 inv_r2 = make_float2(inv_r, inv_r);
             const float2 ngc2 = make_float2(jn.next_gc, jn.next_gc);
-            uint32_t nw2[8], pw[8];
-            if (has) load_block16(jn.next_w + col, nw2);
-            else
-#pragma unroll
-                for (int i = 0; i < 8; ++i) nw2[i] = 0u;
 #pragma unroll
             for (int i = 0; i < 8; ++i) pw[i] = pack_bf16x2_rn(mul2(mul2(r[i], add2(ngc2, unpack_bf16x2(nw2[i]))), inv_r2));
-            if (has) store_block16(jn.next_prenorm + static_cast<size_t>(t) * H + col, pw);
+        }
+        if (has) {
+            if (COMBINE && a.out != nullptr) store_block16(a.out + static_cast<size_t>(t) * H + col, bw);
+            float* rw = jn.residual + static_cast<size_t>(t) * H + col;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<float4*>(rw + 4 * c) =
+                    make_float4(r[2 * c].x, r[2 * c].y, r[2 * c + 1].x, r[2 * c + 1].y);
+            if (jn.next_w != nullptr) store_block16(jn.next_prenorm + static_cast<size_t>(t) * H + col, pw);
         }
     }
     // no CTA leaves while another may still read its shared memory
-    if constexpr (C > 1) cluster_sync_all();
+    if constexpr (C > 1) cluster_exit_sync();
 }
 
 // Threads per CTA and CTAs per cluster for row length H: TPB * C equals the
