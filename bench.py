@@ -4,9 +4,9 @@
 Workload (one step, per GPU): T=8192 tokens, H=8192, E=256 experts, top-8,
 router logits FP32 N(0, 2), 5% of tokens masked, 1% of expert slots invalid,
 expert outputs [T*8, H] BF16 -- synthetic, seeded, resident in HBM.  The
-three calls go through the library's C ABI on one stream (moe_route,
-norm_quant_nvfp4, expert_combine; `--joint` enqueues the first two with the
-single moe_route_norm_quant call).
+calls go through the library's C ABI on one stream: moe_route_norm_quant (the
+router and the pre-expert norm-quant of the same tokens) and expert_combine;
+`--separate` issues moe_route and norm_quant_nvfp4 as two calls instead.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -270,7 +270,7 @@ def run_ours(args, world, rank, local):
 
     def pre_expert():
         # the router gate and the pre-expert RMSNorm + NVFP4 of the same tokens
-        if not args.joint:
+        if args.separate:
             eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
             eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed,
                                 sf=sf)
@@ -454,18 +454,23 @@ def run_decode(eb, dev, reps):
     def nq():
         eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, packed=packed, sf=sf)
 
+    def pre():
+        # the joint call: at this size the router runs beside the norm-quant
+        eb.moe_route_norm_quant(case.logits, case.bias, case.mask, k, case.x, case.norm_w, case.gc,
+                                case.eps, case.gs, topk_ids=ids, topk_weights=w, packed=packed, sf=sf)
+
     def cj():
         eb.expert_combine_join(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                                case.eps, res, case.gain, case.alpha, case.beta, case.eps, case.next_w,
                                case.next_gc, case.eps, out=out, next_prenorm=nxt)
 
     def step():
-        route()
-        nq()
+        pre()
         cj()
 
     r = {"workload": f"decode T={T} H={H} E={case.E} k={k}, join + next prenorm fused",
          "route_us": _graph_us(route, reps, dev), "norm_quant_us": _graph_us(nq, reps, dev),
+         "route_norm_quant_us": _graph_us(pre, reps, dev),
          "combine_join_us": _graph_us(cj, reps, dev), "step_us": _graph_us(step, reps, dev),
          "how": f"{reps} calls per CUDA graph, one replay between two events"}
     r["tokens_per_s"] = T / (r["step_us"] * 1e-6)
@@ -519,8 +524,8 @@ def main():
     ap.add_argument("--no-dispatch", action="store_true",
                     help="skip the separate timing of the dispatch step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--joint", action="store_true",
-                    help="enqueue the pre-expert stages with the joint moe_route_norm_quant call")
+    ap.add_argument("--separate", action="store_true",
+                    help="issue moe_route and norm_quant_nvfp4 as two calls instead of moe_route_norm_quant")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -16,6 +16,13 @@ const DeviceInfo& device_info();   // current device, cached per device
 cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                          int k, int32_t* ids, float* weights, cudaStream_t s);
 
+// The router launched right after the norm-quant of the same tokens, running
+// beside it (see route.cu); used for batches up to kRouteBesideTokensPerSM
+// tokens per SM.
+constexpr int kRouteBesideTokensPerSM = 12;
+cudaError_t launch_route_beside(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
+                                int k, int32_t* ids, float* weights, cudaStream_t s);
+
 cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uint16_t* w, float gc,
                               float eps, const float* gs, uint8_t* packed, uint8_t* sf,
                               cudaStream_t s);

@@ -521,11 +521,19 @@ cudaError_t launch_route_norm_quant(const float* logits, const float* bias, cons
                                     int32_t* ids, float* weights, const uint16_t* x, int M, int H, int tp,
                                     const uint16_t* w, float gc, float eps, const float* gs, uint8_t* packed,
                                     uint8_t* sf, cudaStream_t s) {
-    // The router is latency-bound and wants every warp slot of the SMs, the
-    // norm-quant is streaming-bound and holds their shared memory and most of
-    // their registers; run back to back (programmatic dependent launch
-    // overlaps their edges) they beat any single kernel that splits the SMs
-    // between the two.
+    // The norm-quant is streaming-bound and holds each SM's shared memory
+    // and most of its registers; the router is latency-bound, needs little of
+    // either, but wants many warps in flight.  When its tokens fit one wave of
+    // the warp slots a norm-quant CTA leaves free (three 2-warp CTAs per SM,
+    // two tokens per warp), the norm-quant goes first and the router follows
+    // beside it (programmatic dependent launch lets it start as soon as the
+    // norm-quant kernel is running).  Larger batches run the router first with
+    // every warp slot, then the norm-quant.
+    if (M <= device_info().sm_count * kRouteBesideTokensPerSM) {
+        cudaError_t e = launch_norm_quant(x, M, H, tp, w, gc, eps, gs, packed, sf, s);
+        if (e != cudaSuccess) return e;
+        return launch_route_beside(logits, bias, mask, M, E, k, ids, weights, s);
+    }
     cudaError_t e = launch_route(logits, bias, mask, M, E, k, ids, weights, s);
     if (e != cudaSuccess) return e;
     return launch_norm_quant(x, M, H, tp, w, gc, eps, gs, packed, sf, s);

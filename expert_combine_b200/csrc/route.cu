@@ -330,13 +330,22 @@ __device__ __forceinline__ void route_token_list(const float* l, const float* bi
 
 // MODE > 0: the small path with EPL = MODE scores per lane; MODE < 0: the
 // list path with L = -MODE entries.
-template <int MODE>
+//
+// BESIDE: launched right after the norm-quant kernel of the same tokens, to
+// run in the registers and warp slots that kernel leaves free on every SM.
+// It then starts without waiting for that kernel (it does not read its
+// outputs; the norm-quant kernel lets it launch only after its own wait for
+// the kernels before it, so the router's inputs are ready and the previous
+// readers of ids / weights are done), and waits for it at the end, so that
+// the router finishes after the norm-quant and the kernels after it may rely
+// on both.
+template <int MODE, bool BESIDE>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
                                                     const float* __restrict__ bias,
                                                     const uint8_t* __restrict__ mask, int T, int E,
                                                     int k, int32_t* __restrict__ ids,
                                                     float* __restrict__ weights) {
-    griddep_wait();     // inputs may come from the previous kernel on the stream
+    if constexpr (!BESIDE) griddep_wait();     // inputs may come from the previous kernel on the stream
     griddep_launch();
     const int lane = threadIdx.x & 31;
     const int warp = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
@@ -374,34 +383,50 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
             route_write(l, k, lane, pick_id, id_row, w_row);
         }
     }
+    if constexpr (BESIDE) griddep_wait();
 }
 
-cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
-                         int k, int32_t* ids, float* weights, cudaStream_t s) {
+namespace {
+
+template <bool BESIDE>
+cudaError_t launch_route_cfg(const float* logits, const float* bias, const uint8_t* mask, int T, int E, int k,
+                             int32_t* ids, float* weights, int threads, int grid_cap, cudaStream_t s) {
     const int per_lane = (E + 31) / 32;
-    const int warps_per_cta = 8;
-    const int epl0 = ((E + 31) / 32 + 3) / 4 * 4;
-    const int tokens_per_warp = epl0 <= 16 ? 2 : 1;   // the small path routes two tokens per warp
+    const int warps_per_cta = threads / 32;
+    // scores per lane, rounded up to whole 128-bit loads
+    const int epl = (per_lane + 3) / 4 * 4;
+    const int tokens_per_warp = epl <= 16 ? 2 : 1;   // the small path routes two tokens per warp
     int grid = (T + warps_per_cta * tokens_per_warp - 1) / (warps_per_cta * tokens_per_warp);
-    const int cap = device_info().sm_count * 8;
-    if (grid > cap) grid = cap;
+    if (grid > grid_cap) grid = grid_cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(threads);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // scores per lane, rounded up to whole 128-bit loads
-    const int epl = (per_lane + 3) / 4 * 4;
-    if (epl <= 4) return cudaLaunchKernelEx(&cfg, route_kernel<4>, logits, bias, mask, T, E, k, ids, weights);
-    if (epl <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8>, logits, bias, mask, T, E, k, ids, weights);
-    if (epl <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16>, logits, bias, mask, T, E, k, ids, weights);
-    if (k <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<-8>, logits, bias, mask, T, E, k, ids, weights);
-    if (k <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<-16>, logits, bias, mask, T, E, k, ids, weights);
-    return cudaLaunchKernelEx(&cfg, route_kernel<-32>, logits, bias, mask, T, E, k, ids, weights);
+    if (epl <= 4) return cudaLaunchKernelEx(&cfg, route_kernel<4, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    if (epl <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    if (epl <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    if (k <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<-8, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    if (k <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<-16, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    return cudaLaunchKernelEx(&cfg, route_kernel<-32, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+}
+
+}  // namespace
+
+cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
+                         int k, int32_t* ids, float* weights, cudaStream_t s) {
+    return launch_route_cfg<false>(logits, bias, mask, T, E, k, ids, weights, 256, device_info().sm_count * 8, s);
+}
+
+cudaError_t launch_route_beside(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
+                                int k, int32_t* ids, float* weights, cudaStream_t s) {
+    // 64-thread CTAs, at most three per SM: six warps of 64 registers fit
+    // beside a norm-quant CTA (512 threads x 104 registers)
+    return launch_route_cfg<true>(logits, bias, mask, T, E, k, ids, weights, 64, device_info().sm_count * 3, s);
 }
 
 }  // namespace mb

@@ -287,3 +287,35 @@ def test_full_size_sampled(cuda_dev, name):
                                case.next_gc, case.eps)
         check_join_outputs(synth.host(r)[tokens], synth.host(p)[tokens], r_o, p_o, case.beta)
     assert eb.device_status() == 0
+
+
+@pytest.mark.parametrize("T", [100, 2000])
+def test_joint_pre_expert_steps_feed_the_combine(cuda_dev, T):
+    """Several steps of (moe_route_norm_quant -> expert_combine) on one stream,
+    new logits each step, no synchronisation in between: each step's combine
+    must use that step's routing weights (the router running beside the
+    norm-quant at 100 tokens, before it at 2000)."""
+    case = synth.make_case("tiny", device=cuda_dev, T=T, H=1024, E=64, k=8, join=False)
+    k, H = case.k, case.H
+    ids = torch.empty(T, k, dtype=torch.int32, device=cuda_dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=cuda_dev)
+    packed = torch.empty(T, H // 2, dtype=torch.uint8, device=cuda_dev)
+    sf = torch.empty(T, H // 16, dtype=torch.uint8, device=cuda_dev)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(17)
+    logits_steps = [torch.randn(T, case.E, generator=g).to(cuda_dev) for _ in range(3)]
+    outs = []
+    for lg in logits_steps:
+        case.logits.copy_(lg)
+        eb.moe_route_norm_quant(case.logits, case.bias, case.mask, k, case.x, case.norm_w, case.gc,
+                                case.eps, case.gs, topk_ids=ids, topk_weights=w, packed=packed, sf=sf)
+        outs.append(eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
+                                      case.eps))
+    torch.cuda.synchronize()
+    tokens = sample_tokens(T, 40, seed=T)
+    for lg, out in zip(logits_steps, outs):
+        ids_o, w_o = oracle.route(synth.host(lg), synth.host(case.bias), synth.host(case.mask), k)
+        want = oracle_combine(case, w_o, tokens)
+        got = synth.host(out.index_select(0, torch.as_tensor(tokens, device=cuda_dev)))
+        assert bf16_ulp_diff(got, want).max() <= 1
+    assert eb.device_status() == 0
