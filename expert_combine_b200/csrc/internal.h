@@ -19,7 +19,7 @@ cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* 
 // The router launched right after the norm-quant of the same tokens, running
 // beside it (see route.cu); used for batches up to kRouteBesideTokensPerSM
 // tokens per SM.
-constexpr int kRouteBesideTokensPerSM = 12;
+constexpr int kRouteBesideTokensPerSM = 6;
 cudaError_t launch_route_beside(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                                 int k, int32_t* ids, float* weights, cudaStream_t s);
 

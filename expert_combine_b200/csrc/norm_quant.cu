@@ -525,7 +525,7 @@ cudaError_t launch_route_norm_quant(const float* logits, const float* bias, cons
     // and most of its registers; the router is latency-bound, needs little of
     // either, but wants many warps in flight.  When its tokens fit one wave of
     // the warp slots a norm-quant CTA leaves free (three 2-warp CTAs per SM,
-    // two tokens per warp), the norm-quant goes first and the router follows
+    // one token per warp), the norm-quant goes first and the router follows
     // beside it (programmatic dependent launch lets it start as soon as the
     // norm-quant kernel is running).  Larger batches run the router first with
     // every warp slot, then the norm-quant.

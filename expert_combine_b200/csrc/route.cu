@@ -352,7 +352,27 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
     const bool vec = (E & 3) == 0;
 
-    if constexpr (MODE > 0) {
+    if constexpr (MODE > 0 && BESIDE) {
+        // one token per warp: the shortest chain per token (few tokens, every
+        // warp on an SM sub-partition of its own)
+        for (int t = warp; t < T; t += nwarps) {
+            int32_t* id_row = ids + static_cast<size_t>(t) * k;
+            float* w_row = weights + static_cast<size_t>(t) * k;
+            if (mask[t] == 0) {
+                if (lane < k) {
+                    id_row[lane] = -1;
+                    w_row[lane] = 0.0f;
+                }
+                continue;
+            }
+            const float* l = logits + static_cast<size_t>(t) * E;
+            float lv[MODE];
+            load_logits<MODE>(l, E, lane, vec, lv);
+            uint32_t pick_key = 0u, pick_id = 0u;
+            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+            route_write(l, k, lane, pick_id, id_row, w_row);
+        }
+    } else if constexpr (MODE > 0) {
         // two tokens per iteration: t and t + nwarps
         for (int t = warp; t < T; t += 2 * nwarps) {
             const int tb = t + nwarps;
@@ -395,7 +415,7 @@ cudaError_t launch_route_cfg(const float* logits, const float* bias, const uint8
     const int warps_per_cta = threads / 32;
     // scores per lane, rounded up to whole 128-bit loads
     const int epl = (per_lane + 3) / 4 * 4;
-    const int tokens_per_warp = epl <= 16 ? 2 : 1;   // the small path routes two tokens per warp
+    const int tokens_per_warp = (epl <= 16 && !BESIDE) ? 2 : 1;   // the small path routes two tokens per warp
     int grid = (T + warps_per_cta * tokens_per_warp - 1) / (warps_per_cta * tokens_per_warp);
     if (grid > grid_cap) grid = grid_cap;
     cudaLaunchConfig_t cfg = {};
@@ -425,7 +445,7 @@ cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* 
 cudaError_t launch_route_beside(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                                 int k, int32_t* ids, float* weights, cudaStream_t s) {
     // 64-thread CTAs, at most three per SM: six warps of 64 registers fit
-    // beside a norm-quant CTA (512 threads x 104 registers)
+    // beside a norm-quant CTA (512 threads x 104 registers); one token per warp
     return launch_route_cfg<true>(logits, bias, mask, T, E, k, ids, weights, 64, device_info().sm_count * 3, s);
 }
 

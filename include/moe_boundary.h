@@ -99,7 +99,7 @@ int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* no
  * Source: as moe_route and norm_quant_nvfp4.  The two pre-expert stages read
  * disjoint inputs and are independent (TensorRT-LLM PR 21356, "Where they
  * plug in", runs the pre-expert norm beside the router).  Both kernels are
- * enqueued on `stream`; for small batches (up to 12 tokens per SM) the router
+ * enqueued on `stream`; for small batches (up to 6 tokens per SM) the router
  * runs concurrently with the norm-quant kernel, in the registers and warp
  * slots that kernel leaves free, otherwise the router runs first.  The call
  * completes, in stream order, when both have.  Results are those of the two
