@@ -67,6 +67,7 @@ def _load():
                 "oc_combine": (None, [P, i64, i32, P, P, i32, i32, P, f32, f32, P]),
                 "oc_join": (None, [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32]),
                 "oc_dispatch": (None, [P, i32, i32, i32, i32, P, P, P]),
+                "oc_router_logits": (None, [P, i32, i32, P, i32, f32, P, P]),
                 "oc_bf16_rn_n": (None, [P, i64, P]),
                 "oc_e4m3_rn_sat_n": (None, [P, i64, P]),
                 "oc_e2m1_code_n": (None, [P, i64, P]),
@@ -269,3 +270,21 @@ def dispatch(ids, e0: int, E: int):
     row_token = np.empty(T * k, dtype=np.int32)
     _load().oc_dispatch(_ptr(ids), T, k, e0, E, _ptr(offsets), _ptr(row_idx), _ptr(row_token))
     return offsets, row_idx, row_token
+
+
+def router_logits(x_bf16, W, scale: float = 1.0):
+    """Router projection in binary64 (TensorRT-LLM PR 21356, description,
+    "Router projection": FP32 weights, FP32 accumulation, BF16 input cast,
+    scale folded in).
+
+    ``x_bf16`` uint16 [T, H] (BF16 bits), ``W`` float32 [E, H].  Returns
+    (logits float64 [T, E], abs_sum float64 [T, E]) with abs_sum the sum of
+    |scale * x * W| (the size of the rounding error of an FP32 evaluation)."""
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    T, H = x.shape
+    E = W.shape[0]
+    out = np.empty((T, E), dtype=np.float64)
+    ab = np.empty((T, E), dtype=np.float64)
+    _load().oc_router_logits(_ptr(x), T, H, _ptr(W), E, float(scale), _ptr(out), _ptr(ab))
+    return out, ab

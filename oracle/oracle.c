@@ -23,6 +23,9 @@
  *    _quantize_nvfp4_global_scale and norm_quant_trtllm_nvfp4: per-16 amax,
  *    E4M3 block scale from the global scale, E2M1 thresholds, sign bit,
  *    nibble packing, linear scale layout, the rank-block input layout.
+ *  - TensorRT-LLM PR 21356, description, "Router projection": the router
+ *    logits come from a projection with FP32 weights and FP32 accumulation,
+ *    the BF16 input cast to FP32 and a scale folded in.
  *  - "MoE gate v2" (lmdeploy PR 4835), commit notes: a required token mask;
  *    invalid tokens produce no routing entries; absent rows marked -1; the
  *    gate's routing entries are grouped per expert by a histogram and a scan
@@ -423,6 +426,36 @@ void oc_join(float* residual, const uint16_t* branch, const uint16_t* gain, floa
             oc_norm_row(r, next_w, next_gc, inv2, H, next_prenorm + (size_t)t * H);
         }
         free(g);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Router projection                                                    */
+/* ------------------------------------------------------------------ */
+
+/* x [T, H] BF16 (the hidden states), W [E, H] FP32 (the router weight).
+ *   logits[t, e] = scale * sum_h float(x[t, h]) * W[e, h]
+ * evaluated in binary64: every product of a BF16 and a binary32 value is
+ * exact in binary64, the sum is accumulated in binary64 in h order.  out64
+ * receives the binary64 value, abs64 (if not NULL) the binary64 sum of
+ * |scale * x * W| -- the scale of the rounding error an FP32 evaluation may
+ * make. */
+void oc_router_logits(const uint16_t* x, int T, int H, const float* W, int E, float scale,
+                      double* out64, double* abs64) {
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0, a = 0.0;
+            const uint16_t* xr = x + (size_t)t * H;
+            const float* wr = W + (size_t)e * H;
+            for (int h = 0; h < H; ++h) {
+                double p = (double)oc_bf16_to_f32(xr[h]) * (double)wr[h];
+                s += p;
+                a += fabs(p);
+            }
+            out64[(size_t)t * E + e] = (double)scale * s;
+            if (abs64) abs64[(size_t)t * E + e] = fabs((double)scale) * a;
+        }
     }
 }
 
