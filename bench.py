@@ -468,7 +468,19 @@ def run_decode(eb, dev, reps):
         pre()
         cj()
 
+    # router projection producing this step's logits: x [T, H] BF16, W [E, H] FP32 (seeded)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(synth.SEEDS["decode"] + 7)
+    w_router = (torch.randn(case.E, H, generator=g) / H ** 0.5).to(dev)
+    w3_router = eb.router_weight_prepare(w_router)   # once, when the weight loads
+    logits = torch.empty(T, case.E, dtype=torch.float32, device=dev)
+
+    def proj():
+        eb.router_logits(case.x, w3_router, 1.0, logits=logits)
+
     r = {"workload": f"decode T={T} H={H} E={case.E} k={k}, join + next prenorm fused",
+         "router_logits_us": _graph_us(proj, reps, dev),
+         "router_logits_bytes": case.E * H * 6 + T * H * 2 + T * case.E * 4,
          "route_us": _graph_us(route, reps, dev), "norm_quant_us": _graph_us(nq, reps, dev),
          "route_norm_quant_us": _graph_us(pre, reps, dev),
          "combine_join_us": _graph_us(cj, reps, dev), "step_us": _graph_us(step, reps, dev),

@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     STAGE_NORM_QUANT,
     STAGE_ROUTE,
     STAGE_ROUTE_NORM_QUANT,
+    STAGE_ROUTER_LOGITS,
     device_status,
     dispatch_workspace_size,
     expert_combine,
@@ -32,5 +33,7 @@ from ._lib import (  # noqa: F401
     moe_route_norm_quant,
     norm_quant_nvfp4,
     residual_join,
+    router_logits,
+    router_weight_prepare,
     supported,
 )

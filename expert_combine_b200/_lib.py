@@ -17,6 +17,7 @@ STAGE_JOIN = 3
 STAGE_COMBINE_JOIN = 4
 STAGE_ROUTE_NORM_QUANT = 5
 STAGE_DISPATCH = 6
+STAGE_ROUTER_LOGITS = 7
 
 _lock = threading.Lock()
 _lib = None
@@ -63,6 +64,8 @@ def load() -> ctypes.CDLL:
                                          P, P],
                 "moe_dispatch": [P, i32, i32, i32, i32, P, P, P, P, ctypes.c_size_t, P],
                 "moe_dispatch_noalloc": [P, i32, i32, i32, i32, P, P, P, P],
+                "router_logits": [P, i32, i32, P, i32, f32, P, P],
+                "router_weight_prepare": [P, i32, i32, P, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
                 "mb_last_error": [],
                 "mb_device_status": [],
@@ -360,3 +363,36 @@ def moe_dispatch_noalloc(topk_ids: torch.Tensor, num_experts: int, expert_begin:
            load().moe_dispatch_noalloc(_ptr(topk_ids), T, k, int(expert_begin), E, _ptr(expert_offsets),
                                        _ptr(row_idx), _ptr(row_token), _stream(stream)))
     return expert_offsets, row_idx, row_token
+
+
+def router_weight_prepare(w: torch.Tensor, w3: Optional[torch.Tensor] = None, stream=None):
+    """FP32 router weight [E, H] -> its three BF16 parts [3, E, H] (done once)."""
+    _want(w, torch.float32, "w")
+    E, H = w.shape
+    if w3 is None:
+        w3 = torch.empty(3, E, H, dtype=torch.bfloat16, device=w.device)
+    _want(w3, torch.bfloat16, "w3")
+    if w3.shape != (3, E, H):
+        raise ValueError("router_weight_prepare: shape mismatch")
+    _check("router_weight_prepare", load().router_weight_prepare(_ptr(w), E, H, _ptr(w3), _stream(stream)))
+    return w3
+
+
+def router_logits(x: torch.Tensor, w3: torch.Tensor, scale: float = 1.0,
+                  logits: Optional[torch.Tensor] = None, stream=None):
+    """Router projection on the tensor cores: logits float32 [T, E] =
+    scale * x [T, H] (BF16) @ w^T, w given as its prepared parts w3 [3, E, H]."""
+    _want(x, torch.bfloat16, "x")
+    _want(w3, torch.bfloat16, "w3")
+    T, H = x.shape
+    E = w3.shape[1]
+    if w3.shape != (3, E, H):
+        raise ValueError("router_logits: shape mismatch")
+    if logits is None:
+        logits = torch.empty(T, E, dtype=torch.float32, device=x.device)
+    _want(logits, torch.float32, "logits")
+    if logits.shape != (T, E):
+        raise ValueError("router_logits: shape mismatch")
+    _check("router_logits", load().router_logits(_ptr(x), T, H, _ptr(w3), E, float(scale), _ptr(logits),
+                                                 _stream(stream)))
+    return logits

@@ -72,6 +72,11 @@ int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp) {
             return (hidden_ok(H) && k >= 1 && k <= kMaxTopK) ? 1 : 0;
         case MB_STAGE_JOIN:
             return hidden_ok(H) ? 1 : 0;
+        case MB_STAGE_ROUTER_LOGITS:
+            return (H >= 64 && H % 64 == 0 && H <= kMaxHidden && E >= 16 && E % 16 == 0 && E <= kMaxExperts &&
+                    (static_cast<int64_t>(T) + 127) / 128 <= 65535)
+                       ? 1
+                       : 0;
         case MB_STAGE_DISPATCH:
             return (k >= 1 && k <= kMaxTopK && E >= 1 && E <= kMaxExperts &&
                     static_cast<int64_t>(T) * k <= INT32_MAX)
@@ -222,6 +227,31 @@ int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, con
     return cuda_status(launch_combine(expert_out, num_rows, H, row_idx, weights, T, k, norm_w, gain_center,
                                       eps, out, j, static_cast<cudaStream_t>(stream)),
                        "expert_combine_join");
+}
+
+int router_weight_prepare(const float* w, int E, int H, uint16_t* w3, void* stream) {
+    const char* fn = "router_weight_prepare";
+    if (E < 0 || H < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (!moe_boundary_supported(MB_STAGE_ROUTER_LOGITS, 1, H, E, 0, 1))
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs H %% 64 == 0, 64 <= H <= %d, E %% 16 == 0, 16 <= E <= %d (H=%d, E=%d)",
+                    fn, kMaxHidden, kMaxExperts, H, E);
+    if (!w || !w3) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(w) || !aligned16(w3)) return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return cuda_status(launch_router_weight_split(w, E, H, w3, static_cast<cudaStream_t>(stream)), fn);
+}
+
+int router_logits(const uint16_t* x, int T, int H, const uint16_t* w3, int E, float scale, float* logits,
+                  void* stream) {
+    const char* fn = "router_logits";
+    if (T < 0 || H < 0 || E < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (!moe_boundary_supported(MB_STAGE_ROUTER_LOGITS, T, H, E, 0, 1))
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs H %% 64 == 0, 64 <= H <= %d, E %% 16 == 0, 16 <= E <= %d (H=%d, E=%d)",
+                    fn, kMaxHidden, kMaxExperts, H, E);
+    if (T == 0) return MB_OK;
+    if (!x || !w3 || !logits) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(x) || !aligned16(w3) || !aligned16(logits))
+        return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return cuda_status(launch_router_proj(x, T, H, w3, E, scale, logits, static_cast<cudaStream_t>(stream)), fn);
 }
 
 size_t moe_dispatch_workspace_size(int T, int k, int E) {

@@ -59,6 +59,14 @@ cudaError_t launch_combine_cluster(const uint16_t* expert_out, int64_t R, int H,
                                    uint16_t* out, const JoinArgs& join, cudaStream_t s);
 cudaError_t launch_join_cluster(const uint16_t* branch, int T, int H, const JoinArgs& join, cudaStream_t s);
 
+// Router projection (router_proj.cu): logits = scale * x W^T on the tensor
+// cores from the FP32 weight prepared into three BF16 parts; C K-chunks per
+// expert tile (a cluster of C CTAs).
+int router_proj_chunks(int H);
+cudaError_t launch_router_weight_split(const float* w, int E, int H, uint16_t* w3, cudaStream_t s);
+cudaError_t launch_router_proj(const uint16_t* x, int T, int H, const uint16_t* w3, int E, float scale, float* logits,
+                               cudaStream_t s);
+
 // Dispatch: workspace bytes for n = T * k entries (0 when one tile holds
 // them all), and the launch (one kernel, or three with the workspace).
 size_t dispatch_workspace_bytes(int64_t n, int E);

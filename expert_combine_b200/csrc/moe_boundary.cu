@@ -7,5 +7,6 @@
 #include "route.cu"
 #include "norm_quant.cu"
 #include "decode.cu"
+#include "router_proj.cu"
 #include "dispatch.cu"
 #include "dispatch_noalloc.cu"

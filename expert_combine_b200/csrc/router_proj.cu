@@ -1,0 +1,333 @@
+// router_proj.cu -- the router projection: logits = scale * x W^T with an
+// FP32 router weight, on the 5th-generation tensor cores (tcgen05, BF16
+// operands, FP32 accumulator in tensor memory).
+//
+// TensorRT-LLM PR 21356 "Muse Spark Open decoder fast paths", description,
+// "Router projection": FP32 weights and FP32 accumulation for up to 128
+// tokens, the input cast and a scale folded in, tensor cores with a split of
+// the FP32 operand from 16 tokens (the same page lists a BF16x3 router among
+// its experiments).
+//
+// Precision.  The hidden states are BF16, so x needs no split.  The FP32
+// weight is prepared once into three BF16 parts, w = w1 + w2 + w3 + d with
+// w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2) (each remainder is
+// exact in FP32) and |d| <= 2^-27 |w|.  A product of two BF16 values is exact
+// in FP32, so x W^T = x w1^T + x w2^T + x w3^T, three MMAs per K step,
+// accumulated in FP32 by the tensor core.
+//
+// Work split (one M tile of 128 token rows per grid row; rows >= T read as
+// zero): each CTA owns 16 experts and one of C contiguous K chunks, C <= 8
+// CTAs of a thread-block cluster.  One thread streams the chunk's slabs of
+// 64 K elements with TMA into a 4-stage ring (x: 128 rows x 128 bytes, the
+// three weight parts: 16 rows x 128 bytes each, all 128-byte swizzled, which
+// is the K-major layout the MMA reads); another thread issues each slab's 12
+// MMAs (4 K steps of 16 x 3 parts, M = 128, N = 16) into a 128 x 16 FP32
+// accumulator in tensor memory and hands the stage back with tcgen05.commit.
+// No CTA-wide barrier runs inside the K loop.  The C partial accumulators are
+// then summed across the cluster in rank order through distributed shared
+// memory (no atomics: the same result run to run), scaled, and written for the
+// tokens below T.
+#include "internal.h"
+#include "common.cuh"
+#include "tmap.h"
+
+namespace mb {
+
+namespace {
+
+constexpr int kRpThreads = 128;           // 4 warps: one per tensor-memory lane quadrant
+constexpr int kRpM = 128;                 // token rows per MMA tile
+constexpr int kRpN = 16;                  // experts per CTA (MMA N)
+constexpr int kRpSlabK = 64;              // K elements per slab (one 128-byte swizzle row of BF16)
+constexpr int kRpStages = 4;
+constexpr int kRpXTile = kRpM * 128;      // 16 KB
+constexpr int kRpWTile = kRpN * 128;      // 2 KB per weight part
+constexpr int kRpStageBytes = kRpXTile + 3 * kRpWTile;
+constexpr size_t kRpSmemBytes = 1024 + kRpStages * kRpStageBytes + kRpM * kRpN * 4;
+constexpr int kRpTmemCols = 32;           // allocation unit >= N
+
+struct RouterProjArgs {
+    float* logits;        // [T, E] FP32
+    int T, H, E;
+    int kc;               // K elements per CTA (a multiple of 64)
+    float scale;
+};
+
+// ---- tcgen05 / tensor-memory primitives (cta_group::1)
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[128 x N] (+)= A[128 x 16] B[N x 16]^T, BF16 operands from shared memory.
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+// Arrive on `bar` once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+// 16 consecutive FP32 columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups
+// 1024 bytes apart (stride byte offset), leading byte offset unused (1),
+// descriptor version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1u) << 16) |
+           (static_cast<uint64_t>(1024u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46) |
+           (static_cast<uint64_t>(2u) << 61);
+}
+
+// Instruction descriptor: FP32 accumulator, BF16 A and B, both K-major,
+// N = kRpN, M = kRpM.
+constexpr uint32_t kRpIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kRpN >> 3) << 17) |
+                              (static_cast<uint32_t>(kRpM >> 4) << 24);
+
+template <int C>
+__global__ void __launch_bounds__(kRpThreads) router_proj_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                 const __grid_constant__ CUtensorMap wmap,
+                                                                 const RouterProjArgs a) {
+    extern __shared__ uint8_t rp_smem_raw[];
+    const uint32_t raw = smem_addr(rp_smem_raw);
+    uint8_t* stages = rp_smem_raw + (((raw + 1023u) & ~1023u) - raw);   // 1024-byte aligned (128-byte swizzle)
+    float* part = reinterpret_cast<float*>(stages + kRpStages * kRpStageBytes);   // [128][16] partial sums
+    __shared__ __align__(8) uint64_t full[kRpStages];    // slab landed (TMA)
+    __shared__ __align__(8) uint64_t empty[kRpStages];   // slab's MMAs done (tcgen05.commit)
+    __shared__ __align__(8) uint64_t done;               // every MMA done
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_issued, s_consumed;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int krank = blockIdx.x % C;
+    const int e0 = (blockIdx.x / C) * kRpN;
+    const int m0 = blockIdx.y * kRpM;
+    const int kbase = krank * a.kc;
+    const int J = a.kc / kRpSlabK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRpStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(&done, 1);
+        s_issued = 0;
+        s_consumed = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, kRpTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = s_tmem;
+    griddep_wait();
+    griddep_launch();
+
+    // One lane of warp 0 produces, one lane of warp 1 issues the MMAs; their
+    // warp-mates wait at __syncwarp (not on the barriers, which would make the
+    // whole warp sleep with them).
+    if (warp == 0) {
+        if (lane == 0) {                // TMA producer
+        int j = 0;
+        for (; j < J; ++j) {
+            const int s = j % kRpStages;
+            if (j >= kRpStages && !mbar_wait_bounded(&empty[s], static_cast<uint32_t>((j / kRpStages - 1) & 1), 8u))
+                break;
+            uint8_t* st = stages + s * kRpStageBytes;
+            const int k0 = kbase + j * kRpSlabK;
+            mbar_arrive_expect_tx(&full[s], kRpStageBytes);
+            tma_load_2d(smem_addr(st), &xmap, k0, m0, &full[s]);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+                tma_load_2d(smem_addr(st + kRpXTile + p * kRpWTile), &wmap, k0, p * a.E + e0, &full[s]);
+        }
+        s_issued = j;
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {                // MMA issuer
+        int j = 0;
+        for (; j < J; ++j) {
+            const int s = j % kRpStages;
+            if (!mbar_wait_bounded(&full[s], static_cast<uint32_t>((j / kRpStages) & 1), 8u)) break;
+            tc_fence_after();
+            const uint32_t sa = smem_addr(stages + s * kRpStageBytes);
+#pragma unroll
+            for (int ks = 0; ks < kRpSlabK / 16; ++ks) {   // K steps of 16 BF16 = 32 bytes
+                const uint64_t ad = smem_desc_sw128(sa + 32u * ks);
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+                    mma_bf16(tmem_d, ad, smem_desc_sw128(sa + kRpXTile + p * kRpWTile + 32u * ks), kRpIdesc,
+                             (j | ks | p) != 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
+        }
+        s_consumed = j;
+        mma_commit(&done);   // arrives once every MMA issued above has completed
+        }
+        __syncwarp();
+    }
+    const bool finished = mbar_wait_bounded(&done, 0u, 8u);
+    __syncthreads();
+    const bool complete = finished && s_consumed == J;
+    if (threadIdx.x == 0)   // copies issued but never consumed (an early stop) land before the CTA exits
+        for (int j = s_consumed; j < s_issued; ++j)
+            mbar_wait_bounded(&full[j % kRpStages], static_cast<uint32_t>((j / kRpStages) & 1), 8u);
+    tc_fence_after();
+
+    // partial accumulator: warp w holds token rows 32w .. 32w + 31
+    float v[16];
+    tmem_ld16(tmem_d + (static_cast<uint32_t>(32 * warp) << 16), v);
+#pragma unroll
+    for (int n = 0; n < kRpN; ++n) part[(32 * warp + lane) * kRpN + n] = complete ? v[n] : 0.0f;
+    tc_fence_before();
+    if constexpr (C > 1) {
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    } else {
+        __syncthreads();
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_d, kRpTmemCols);
+    }
+
+    // this CTA's rows of the tile: the C partials summed in rank order
+    constexpr int kRows = kRpM / C;
+    for (int o = threadIdx.x; o < kRows * kRpN; o += kRpThreads) {
+        const int m = krank * kRows + o / kRpN, n = o % kRpN;
+        const float* src = part + m * kRpN + n;
+        float pv[C];
+#pragma unroll
+        for (int q = 0; q < C; ++q) {
+            if constexpr (C == 1) {
+                pv[q] = *src;
+            } else {
+                uint32_t remote;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(src)), "r"(q));
+                asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv[q]) : "r"(remote) : "memory");
+            }
+        }
+        const float sum = tree_sum_array<C>(pv);
+        if (m0 + m < a.T) a.logits[static_cast<size_t>(m0 + m) * a.E + e0 + n] = __fmul_rn(a.scale, sum);
+    }
+    if constexpr (C > 1)
+        asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+
+// w3[p][e][h], p = 0, 1, 2: the BF16 parts of w (see the file comment).
+__global__ void router_weight_split_kernel(const float* __restrict__ w, int64_t n, uint16_t* __restrict__ w3) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float x = w[i];
+        const uint16_t b1 = bf16_bits_rn(x);
+        const float r1 = __fsub_rn(x, __uint_as_float(static_cast<uint32_t>(b1) << 16));
+        const uint16_t b2 = bf16_bits_rn(r1);
+        const float r2 = __fsub_rn(r1, __uint_as_float(static_cast<uint32_t>(b2) << 16));
+        w3[i] = b1;
+        w3[n + i] = b2;
+        w3[2 * n + i] = bf16_bits_rn(r2);
+    }
+}
+
+template <int C>
+cudaError_t launch_rp(const CUtensorMap& xmap, const CUtensorMap& wmap, const RouterProjArgs& a, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(router_proj_kernel<C>),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kRpSmemBytes));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((a.E / kRpN) * C, (a.T + kRpM - 1) / kRpM);
+    cfg.blockDim = dim3(kRpThreads);
+    cfg.dynamicSmemBytes = kRpSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if constexpr (C > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = C;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    return cudaLaunchKernelEx(&cfg, router_proj_kernel<C>, xmap, wmap, a);
+}
+
+}  // namespace
+
+// K chunks per expert tile: the largest C in {8, 4, 2, 1} with H % (64 C) == 0.
+int router_proj_chunks(int H) {
+    for (int c = 8; c > 1; c >>= 1)
+        if (H % (kRpSlabK * c) == 0) return c;
+    return 1;
+}
+
+cudaError_t launch_router_weight_split(const float* w, int E, int H, uint16_t* w3, cudaStream_t s) {
+    const int64_t n = static_cast<int64_t>(E) * H;
+    int grid = static_cast<int>((n + 255) / 256);
+    if (grid > device_info().sm_count * 8) grid = device_info().sm_count * 8;
+    router_weight_split_kernel<<<grid, 256, 0, s>>>(w, n, w3);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_proj(const uint16_t* x, int T, int H, const uint16_t* w3, int E, float scale, float* logits,
+                               cudaStream_t s) {
+    const int C = router_proj_chunks(H);
+    const RouterProjArgs a{logits, T, H, E, H / C, scale};
+    CUtensorMap xmap, wmap;
+    if (!encode_2d_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H),
+                       static_cast<uint64_t>(H) * 2, kRpM, kRpSlabK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w3, static_cast<uint64_t>(3) * E,
+                       static_cast<uint64_t>(H), static_cast<uint64_t>(H) * 2, kRpN, kRpSlabK,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    switch (C) {
+        case 8: return launch_rp<8>(xmap, wmap, a, s);
+        case 4: return launch_rp<4>(xmap, wmap, a, s);
+        case 2: return launch_rp<2>(xmap, wmap, a, s);
+        default: return launch_rp<1>(xmap, wmap, a, s);
+    }
+}
+
+}  // namespace mb

@@ -180,6 +180,47 @@ int expert_combine_join(const uint16_t* expert_out, int64_t num_rows, int H, con
                         uint16_t* next_prenorm, void* stream);
 
 /*
+ * router_weight_prepare -- the FP32 router weight in the form router_logits
+ * reads: three BF16 parts of each weight (done once, when the weight loads).
+ *
+ * Source: TensorRT-LLM PR 21356, description, "Router projection" (FP32
+ * weights on tensor cores with a split of the FP32 operand; the page lists a
+ * BF16x3 router among its experiments).
+ *
+ *   w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2)   (round to
+ *   nearest even; each remainder is exact in FP32), |w - w1 - w2 - w3| <=
+ *   2^-27 |w|.
+ *
+ *   w    [E, H] FP32 (row e: expert e)
+ *   w3   [3, E, H] BF16 (out): w1, then w2, then w3; 6 * E * H bytes
+ * Supported: as router_logits.
+ */
+int router_weight_prepare(const float* w, int E, int H, uint16_t* w3, void* stream);
+
+/*
+ * router_logits -- the router projection: logits = scale * x W^T.
+ *
+ * Source: TensorRT-LLM PR 21356, description, "Router projection" (FP32
+ * weights and FP32 accumulation for up to 128 tokens, the input cast and a
+ * scale folded in, tensor cores from 16 tokens).
+ *
+ *   logits[t, e] = scale * sum_h float(x[t, h]) * w[e, h]
+ *
+ * computed on the tensor cores from the prepared weight: x w1^T + x w2^T +
+ * x w3^T with BF16 operands (every product exact in FP32) accumulated in FP32
+ * in a fixed order, so results are reproducible run to run.  The error against
+ * the exact sum is below (2^-27 + (3 H / C / 16 + 12) * 2^-23) *
+ * sum_h |scale * x * w|, with C = 8, 4, 2 or 1 the largest such that
+ * H % (64 C) == 0.
+ *
+ *   x       [T, H] BF16          w3      [3, E, H] BF16 from router_weight_prepare
+ *   logits  [T, E] FP32 (out)
+ * Supported: H % 64 == 0, 64 <= H <= 16384, E % 16 == 0, 16 <= E <= 4096.
+ */
+int router_logits(const uint16_t* x, int T, int H, const uint16_t* w3, int E, float scale, float* logits,
+                  void* stream);
+
+/*
  * moe_dispatch -- expert-grouped rows of the routing entries: the dispatch
  * step between the router (moe_route) and the experts, producing the
  * row_idx that expert_combine reads.
@@ -253,6 +294,7 @@ enum {
     MB_STAGE_COMBINE_JOIN = 4,
     MB_STAGE_ROUTE_NORM_QUANT = 5,
     MB_STAGE_DISPATCH = 6,
+    MB_STAGE_ROUTER_LOGITS = 7,
 };
 
 /*
@@ -269,7 +311,8 @@ const char* mb_last_error(void);
  * mb_device_status -- reads and clears the device-side status word of the
  * current device (synchronous).  Bit 0: a producer's bounded wait for a free
  * shared-memory slot ran out; bit 1: a drain wait ran out; bit 2: a
- * consumer's wait for a copied row ran out.  0 means no kernel reported a
+ * consumer's wait for a copied row ran out; bit 3: the router projection's
+ * wait for its tensor-core MMAs ran out.  0 means no kernel reported a
  * timeout since the last call.  Returns -1 (and sets mb_last_error) when the
  * CUDA runtime fails.
  */

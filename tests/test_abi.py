@@ -22,6 +22,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for fn in ("moe_route", "norm_quant_nvfp4", "expert_combine", "residual_join",
                "expert_combine_join", "moe_dispatch", "moe_dispatch_workspace_size",
+               "router_logits", "router_weight_prepare",
                "moe_boundary_supported", "mb_last_error", "mb_device_status"):
         assert fn in names
 
@@ -49,6 +50,10 @@ def test_supported_predicate():
     assert not eb.supported(eb.STAGE_DISPATCH, 8, 0, 0, 8)
     assert not eb.supported(eb.STAGE_DISPATCH, 8, 0, 4097, 8)
     assert not eb.supported(eb.STAGE_DISPATCH, 1 << 27, 0, 256, 32)
+    assert eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 8192, 256)
+    assert eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 4096, 2560)
+    assert not eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 8200, 256)
+    assert not eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 8192, 250)
     assert not eb.supported(99, 8, 16)
 
 
@@ -85,6 +90,21 @@ def test_bad_arguments_are_rejected_before_any_launch():
     assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, a, ctypes.c_size_t(need - 1), N) == 1
     assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, odd, ctypes.c_size_t(need), N) == 1
     assert "aligned" in eb.last_error()
+
+
+def test_router_projection_arguments_checked_before_launch():
+    lib = eb.load()
+    N = None
+    a = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1004)
+    assert lib.router_logits(N, 4, 8200, N, 256, 1.0, N, N) == 2
+    assert lib.router_logits(N, -1, 8192, N, 256, 1.0, N, N) == 1
+    assert lib.router_logits(N, 0, 8192, N, 256, 1.0, N, N) == 0          # empty: no launch
+    assert lib.router_logits(N, 4, 8192, N, 256, 1.0, N, N) == 1
+    assert lib.router_logits(a, 4, 8192, odd, 256, 1.0, a, N) == 1
+    assert "aligned" in eb.last_error()
+    assert lib.router_weight_prepare(N, 256, 8192, N, N) == 1
+    assert lib.router_weight_prepare(a, 250, 8192, a, N) == 2
 
 
 def test_dispatch_workspace_size():
