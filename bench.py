@@ -37,6 +37,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from expert_combine_b200 import shard  # noqa: E402
+
 WORKLOAD = "prefill"
 METRIC = "tokens/s of route+norm-quant+combine at 8192 tok, H=8192; HBM GB/s vs 8 TB/s"
 NOMINAL_HBM_GBS = 8000.0
@@ -127,34 +129,6 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def init_dist():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 # ---------------------------------------------------------------------------- CPU oracle
 def oracle_step(case_host, tokens):
     """The oracle on a sample of the workload's tokens (all three stages)."""
@@ -216,8 +190,8 @@ def time_oracle(case_host, tokens, budget_s=15.0):
 
 
 # ---------------------------------------------------------------------------- reference arm
-def run_reference(args, world, rank):
-    if rank != 0:
+def run_reference(args, info):
+    if info.rank != 0:
         return 0
     from expert_combine_b200 import synth
     case = synth.make_case(WORKLOAD, device="cuda" if torch.cuda.is_available() else "cpu")
@@ -251,14 +225,15 @@ def run_reference(args, world, rank):
 
 
 # ---------------------------------------------------------------------------- our arm
-def run_ours(args, world, rank, local):
+def run_ours(args, info):
+    world, rank, local = info.world, info.rank, info.local
     import expert_combine_b200 as eb
     from expert_combine_b200 import synth
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     eb.load()
-    case = synth.make_case(WORKLOAD, device=dev, seed=synth.SEEDS[WORKLOAD] + rank,
+    case = synth.make_case(WORKLOAD, device=dev, seed=shard.rank_seed(synth.SEEDS[WORKLOAD], info),
                            T=args.tokens)
     T, H, E, k = case.T, case.H, case.E, case.k
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
@@ -304,7 +279,7 @@ def run_ours(args, world, rank, local):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    barrier(world)
+    shard.barrier(info)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
         time.sleep(0.3)
@@ -312,7 +287,7 @@ def run_ours(args, world, rank, local):
         e0, e1 = timed(step, args.steps)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
-    barrier(world)
+    shard.barrier(info)
     step_ms = e0.elapsed_time(e1)
     # each stage alone, back to back, for the per-kernel launch durations
     pre_ev = timed(pre_expert, args.steps)
@@ -321,7 +296,7 @@ def run_ours(args, world, rank, local):
     stage_ms = [pre_ev[0].elapsed_time(pre_ev[1]) / args.steps,
                 cmb_ev[0].elapsed_time(cmb_ev[1]) / args.steps]
     combine_ms = stage_ms[1]
-    step_ms_max = max_over_ranks(step_ms, world)
+    step_ms_max = shard.max_over_ranks(step_ms, info)
     ms_per_step = step_ms_max / args.steps
 
     # algorithmic bytes
@@ -342,7 +317,7 @@ def run_ours(args, world, rank, local):
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
                                            pre_expert, steps=max(2, min(args.steps, 5)))
 
-    tokens_per_s = T * world / (ms_per_step * 1e-3)
+    tokens_per_s = shard.weak_scaling_throughput(T, ms_per_step, info)
     result = None
     if rank == 0:
         cpu = None
@@ -543,17 +518,16 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    world, rank, local = init_dist() if args.impl == "ours" else (
-        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    # the reference arm runs on rank 0 alone and joins no process group
+    info = shard.init("nccl") if args.impl == "ours" else shard.rank_info()
     try:
         if args.impl == "reference":
-            return run_reference(args, world, rank)
-        run_ours(args, world, rank, local)
+            return run_reference(args, info)
+        run_ours(args, info)
         return 0
     finally:
-        if world > 1 and args.impl == "ours":
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        if args.impl == "ours":
+            shard.finalize(info)
 
 
 if __name__ == "__main__":
