@@ -254,6 +254,8 @@ def run_ours(args, info):
                                     case.gc, case.eps, case.gs, topk_ids=ids, topk_weights=w,
                                     packed=packed, sf=sf)
 
+    pre_kernels = 2 if args.separate else eb.route_norm_quant_kernels(T, H, E, k, tp=case.tp)
+
     def combine():
         eb.expert_combine(case.expert_out, case.R, case.row_idx, w, case.post_w, case.post_gc,
                           case.eps, out=out)
@@ -355,7 +357,7 @@ def run_ours(args, info):
             "e2e": e2e,
             "dispatch": disp,
             "decode": dec,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (pre_kernels + 1) * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
                        "timed_wall_s": t_wall},

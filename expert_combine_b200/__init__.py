@@ -33,6 +33,7 @@ from ._lib import (  # noqa: F401
     moe_route_norm_quant,
     norm_quant_nvfp4,
     residual_join,
+    route_norm_quant_kernels,
     router_logits,
     router_weight_prepare,
     supported,

@@ -67,6 +67,7 @@ def load() -> ctypes.CDLL:
                 "router_logits": [P, i32, i32, P, i32, f32, P, P],
                 "router_weight_prepare": [P, i32, i32, P, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
+                "moe_route_norm_quant_kernels": [i32, i32, i32, i32, i32],
                 "mb_last_error": [],
                 "mb_device_status": [],
             }
@@ -212,6 +213,12 @@ def moe_route_norm_quant(logits: torch.Tensor, bias: torch.Tensor, token_mask: t
                                        _ptr(global_scale), _ptr(packed), _ptr(sf), _stream(stream)))
     return topk_ids, topk_weights, packed, sf
 
+
+
+def route_norm_quant_kernels(M: int, H: int, E: int, k: int, tp: int = 1) -> int:
+    """Kernels ``moe_route_norm_quant`` enqueues for these sizes on the current
+    device (for a 16-byte-aligned x); -1 when unsupported or without a device."""
+    return int(load().moe_route_norm_quant_kernels(M, H, tp, E, k))
 
 def expert_combine(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
                    weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,

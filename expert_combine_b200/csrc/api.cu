@@ -156,6 +156,17 @@ int moe_route_norm_quant(const float* logits, const float* bias, const uint8_t* 
                        "moe_route_norm_quant");
 }
 
+int moe_route_norm_quant_kernels(int M, int H, int tp, int E, int k) {
+    if (!moe_boundary_supported(MB_STAGE_ROUTE_NORM_QUANT, M, H, E, k, tp)) return -1;
+    if (M == 0) return 0;
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || n == 0) {
+        cudaGetLastError();
+        return -1;
+    }
+    return route_norm_quant_kernels(M, H, tp, E);
+}
+
 static int check_combine(const char* fn, const uint16_t* expert_out, int64_t num_rows, int H,
                          const int32_t* row_idx, const float* weights, int T, int k,
                          const uint16_t* norm_w) {

@@ -27,6 +27,8 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
                               float eps, const float* gs, uint8_t* packed, uint8_t* sf,
                               cudaStream_t s);
 
+// Kernels launch_route_norm_quant enqueues for these sizes (x 16-byte aligned).
+int route_norm_quant_kernels(int M, int H, int tp, int E);
 cudaError_t launch_route_norm_quant(const float* logits, const float* bias, const uint8_t* mask, int E, int k,
                                     int32_t* ids, float* weights, const uint16_t* x, int M, int H, int tp,
                                     const uint16_t* w, float gc, float eps, const float* gs, uint8_t* packed,

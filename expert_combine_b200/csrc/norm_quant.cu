@@ -14,6 +14,7 @@
 // layout [tp, M, H/tp] (tp copies per row into one slot).
 #include "internal.h"
 #include "ring.cuh"
+#include "route.cuh"
 #include "tmap.h"
 
 namespace mb {
@@ -28,6 +29,23 @@ struct NormQuantArgs {
     uint8_t* sf;
     int nslot;
 };
+
+// The router's arguments when the wide norm-quant kernel also routes its tokens.
+struct FusedRouteArgs {
+    const float* logits;
+    const float* bias;
+    const uint8_t* mask;
+    int E, k;
+    int32_t* ids;
+    float* weights;
+};
+
+// Router warps added to a wide norm-quant CTA (after its 16 row warps), two
+// per SM sub-partition; at 768 threads the kernel fits in 80 registers a
+// thread without spilling.
+constexpr int kFusedRouterWarps = 8;
+// The router warps use the small selection path with 8 scores per lane.
+constexpr int kFusedRouteMaxExperts = 256;
 
 template <int TW, bool SWZ, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
@@ -168,8 +186,9 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 float q[16];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    // + 0 turns a -0 product into +0 (no sign bit for -0)
-                    const float2 q2 = add2(mul2(unpack_bf16x2(yw[i]), os2), zero2);
+                    // y * os + 0 in one rounding: a -0 product becomes +0 (no sign
+                    // bit for -0), any other product is rounded once as by a multiply
+                    const float2 q2 = fma2(unpack_bf16x2(yw[i]), os2, zero2);
                     q[2 * i] = q2.x;
                     q[2 * i + 1] = q2.y;
                 }
@@ -194,9 +213,17 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // keeps its 32 words in registers across the team barrier, so the slot is
 // refilled as soon as the barrier has passed.  The packed BF16 weights sit in
 // a shared-memory table read without bank conflicts.
-template <int TW, bool GC0>
-__global__ void __launch_bounds__(kConsumerThreads, 1)
-    norm_quant_wide_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a) {
+//
+// ROUTE: the CTA carries router warps after its row warps; they route the same
+// M tokens (two per warp iteration, statically interleaved over the grid's
+// router warps) in the issue slots and registers the streaming row warps
+// leave free, so the latency-bound router adds little to the bandwidth-bound
+// norm-quant.  The router warps touch no shared memory and no barrier after
+// the CTA's set-up.
+template <int TW, bool GC0, bool ROUTE>
+__global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterWarps : 0), 1)
+    norm_quant_wide_kernel(const __grid_constant__ CUtensorMap tmap, const NormQuantArgs a,
+                           const FusedRouteArgs ra) {
     constexpr int P = TW * 32;
     constexpr int NTEAM = kConsumerThreads / P;
     extern __shared__ uint8_t smem_raw[];
@@ -233,6 +260,15 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                                          : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
+    if constexpr (ROUTE) {
+        constexpr int RW = kFusedRouterWarps;
+        if (warp >= NTEAM * TW) {
+            route_pairs<8>(ra.logits, ra.bias, ra.mask, a.M, ra.E, ra.k, ra.ids, ra.weights,
+                           static_cast<int>(blockIdx.x) * RW + (warp - NTEAM * TW),
+                           static_cast<int>(gridDim.x) * RW, lane);
+            return;
+        }
+    }
 
     const int M = a.M;
     const int team_stride = gridDim.x * NTEAM;
@@ -349,7 +385,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
             float q[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float2 q2 = add2(mul2(unpack_bf16x2(yw[i]), os2), zero2);   // -0 -> +0
+                const float2 q2 = fma2(unpack_bf16x2(yw[i]), os2, zero2);   // -0 -> +0, one rounding
                 q[2 * i] = q2.x;
                 q[2 * i + 1] = q2.y;
             }
@@ -413,8 +449,9 @@ cudaError_t launch_nq_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a
     }
 }
 
-template <int TW, bool GC0>
-cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, cudaStream_t s) {
+template <int TW, bool GC0, bool ROUTE>
+cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, const FusedRouteArgs& ra,
+                           cudaStream_t s) {
     constexpr int P = TW * 32;
     constexpr int NTEAM = kConsumerThreads / P;
     const int slot_bytes = slot_bytes_for(args.H);
@@ -428,7 +465,7 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     NormQuantArgs a = args;
     a.nslot = nslot;
     const size_t smem = lay.total_bytes();
-    auto kern = norm_quant_wide_kernel<TW, GC0>;
+    auto kern = norm_quant_wide_kernel<TW, GC0, ROUTE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -437,7 +474,7 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     if (grid > cap) grid = cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kConsumerThreads);
+    cfg.blockDim = dim3(kConsumerThreads + (ROUTE ? 32 * kFusedRouterWarps : 0));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -445,22 +482,26 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmap, a);
+    return cudaLaunchKernelEx(&cfg, kern, tmap, a, ra);
 }
 
-template <bool GC0>
-cudaError_t launch_nq_wide_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
+template <bool GC0, bool ROUTE>
+cudaError_t launch_nq_wide_tw(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, const FusedRouteArgs& ra,
+                              cudaStream_t s) {
     switch (TW) {
-        case 1: return launch_nq_wide<1, GC0>(tmap, a, s);
-        case 2: return launch_nq_wide<2, GC0>(tmap, a, s);
-        case 4: return launch_nq_wide<4, GC0>(tmap, a, s);
-        case 8: return launch_nq_wide<8, GC0>(tmap, a, s);
+        case 1: return launch_nq_wide<1, GC0, ROUTE>(tmap, a, ra, s);
+        case 2: return launch_nq_wide<2, GC0, ROUTE>(tmap, a, ra, s);
+        case 4: return launch_nq_wide<4, GC0, ROUTE>(tmap, a, ra, s);
+        case 8: return launch_nq_wide<8, GC0, ROUTE>(tmap, a, ra, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_nq_wide_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, cudaStream_t s) {
-    return a.gc == 0.0f ? launch_nq_wide_tw<true>(TW, tmap, a, s) : launch_nq_wide_tw<false>(TW, tmap, a, s);
+template <bool ROUTE>
+cudaError_t launch_nq_wide_gc(int TW, const CUtensorMap& tmap, const NormQuantArgs& a, const FusedRouteArgs& ra,
+                              cudaStream_t s) {
+    return a.gc == 0.0f ? launch_nq_wide_tw<true, ROUTE>(TW, tmap, a, ra, s)
+                        : launch_nq_wide_tw<false, ROUTE>(TW, tmap, a, ra, s);
 }
 
 // gc == +0 or -0: the gain is the BF16 weight itself (0 + w == w exactly)
@@ -483,13 +524,18 @@ int team_warps(int H) {
 
 namespace {
 
+// The sizes the wide tensor-map norm-quant path takes.
+bool wide_nq_sizes(int M, int H, int tp) {
+    const int hs = H / tp;
+    return (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
+           static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31) && H >= 2048;
+}
+
 // Tensor map and team width of the norm-quant row copies; false when the
 // wide tensor-map path does not apply.
 bool wide_nq_plan(const uint16_t* x, int M, int H, int tp, CUtensorMap& tmap, int& TW) {
     const int hs = H / tp;
-    const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
-                     static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
-    if (!swz || H < 2048) return false;
+    if (!wide_nq_sizes(M, H, tp)) return false;
     if (!encode_line_map(&tmap, x, static_cast<uint64_t>(M) * tp * (hs / 64), static_cast<uint32_t>(hs / 64)))
         return false;
     int P = 32;
@@ -506,7 +552,7 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
     NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
     CUtensorMap tmap;
     int TW = 0;
-    if (wide_nq_plan(x, M, H, tp, tmap, TW)) return launch_nq_wide_gc(TW, tmap, a, s);
+    if (wide_nq_plan(x, M, H, tp, tmap, TW)) return launch_nq_wide_gc<false>(TW, tmap, a, FusedRouteArgs{}, s);
     const int hs = H / tp;
     const bool swz = (hs % 64 == 0) && (tp == 1 || (2 * hs) % kSlotAlign == 0) &&
                      static_cast<uint64_t>(M) * tp * (hs / 64) < (1ull << 31);
@@ -515,6 +561,13 @@ cudaError_t launch_norm_quant(const uint16_t* x, int M, int H, int tp, const uin
         return launch_nq_gc<true>(team_warps(H), tmap, a, s);
     std::memset(&tmap, 0, sizeof(tmap));
     return launch_nq_gc<false>(team_warps(H), tmap, a, s);
+}
+
+bool route_beside_norm_quant(int M) { return M <= device_info().sm_count * kRouteBesideTokensPerSM; }
+
+int route_norm_quant_kernels(int M, int H, int tp, int E) {
+    if (route_beside_norm_quant(M)) return 2;
+    return (E <= kFusedRouteMaxExperts && wide_nq_sizes(M, H, tp)) ? 1 : 2;
 }
 
 cudaError_t launch_route_norm_quant(const float* logits, const float* bias, const uint8_t* mask, int E, int k,
@@ -527,12 +580,20 @@ cudaError_t launch_route_norm_quant(const float* logits, const float* bias, cons
     // the warp slots a norm-quant CTA leaves free (three 2-warp CTAs per SM,
     // one token per warp), the norm-quant goes first and the router follows
     // beside it (programmatic dependent launch lets it start as soon as the
-    // norm-quant kernel is running).  Larger batches run the router first with
-    // every warp slot, then the norm-quant.
-    if (M <= device_info().sm_count * kRouteBesideTokensPerSM) {
+    // norm-quant kernel is running).  Larger batches on the wide norm-quant
+    // path (E <= 256) route in extra warps of the norm-quant kernel itself;
+    // the rest run the router first with every warp slot, then the norm-quant.
+    if (route_beside_norm_quant(M)) {
         cudaError_t e = launch_norm_quant(x, M, H, tp, w, gc, eps, gs, packed, sf, s);
         if (e != cudaSuccess) return e;
         return launch_route_beside(logits, bias, mask, M, E, k, ids, weights, s);
+    }
+    CUtensorMap tmap;
+    int TW = 0;
+    if (E <= kFusedRouteMaxExperts && wide_nq_plan(x, M, H, tp, tmap, TW)) {
+        const NormQuantArgs a{x, M, H, tp, w, gc, eps, gs, packed, sf, 0};
+        const FusedRouteArgs ra{logits, bias, mask, E, k, ids, weights};
+        return launch_nq_wide_gc<true>(TW, tmap, a, ra, s);
     }
     cudaError_t e = launch_route(logits, bias, mask, M, E, k, ids, weights, s);
     if (e != cudaSuccess) return e;

@@ -98,17 +98,29 @@ int norm_quant_nvfp4(const uint16_t* x, int M, int H, int tp, const uint16_t* no
  *
  * Source: as moe_route and norm_quant_nvfp4.  The two pre-expert stages read
  * disjoint inputs and are independent (TensorRT-LLM PR 21356, "Where they
- * plug in", runs the pre-expert norm beside the router).  Both kernels are
- * enqueued on `stream`; for small batches (up to 6 tokens per SM) the router
- * runs concurrently with the norm-quant kernel, in the registers and warp
- * slots that kernel leaves free, otherwise the router runs first.  The call
- * completes, in stream order, when both have.  Results are those of the two
- * calls with T = M, bit for bit.  Supported: both calls' rules.
+ * plug in", runs the pre-expert norm beside the router).  The work is
+ * enqueued on `stream` in one of three arrangements: for small batches (up to
+ * 6 tokens per SM) the router kernel runs concurrently with the norm-quant
+ * kernel, in the registers and warp slots that kernel leaves free; for larger
+ * batches on the wide norm-quant path (H >= 2048, H / tp % 64 == 0, E <= 256)
+ * one kernel does both, its router warps beside its row warps; otherwise the
+ * router kernel runs first.  The call completes, in stream order, when both
+ * stages have.  Results are those of the two calls with T = M, bit for bit.
+ * Supported: both calls' rules.
  */
 int moe_route_norm_quant(const float* logits, const float* bias, const uint8_t* token_mask, int E, int k,
                          int32_t* topk_ids, float* topk_weights, const uint16_t* x, int M, int H, int tp,
                          const uint16_t* norm_w, float gain_center, float eps, const float* global_scale,
                          uint8_t* packed, uint8_t* sf, void* stream);
+
+/*
+ * moe_route_norm_quant_kernels -- how many kernels moe_route_norm_quant
+ * enqueues for these sizes on the current device (1 or 2), for an input x
+ * whose address is 16-byte aligned (an unaligned x takes a two-kernel
+ * arrangement); 0 for M == 0.  Returns -1 when the sizes are not supported or
+ * no CUDA device is present.  No device work.
+ */
+int moe_route_norm_quant_kernels(int M, int H, int tp, int E, int k);
 
 /*
  * expert_combine -- post-expert RMSNorm of each selected row + weighted sum.

@@ -22,7 +22,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for fn in ("moe_route", "norm_quant_nvfp4", "expert_combine", "residual_join",
                "expert_combine_join", "moe_dispatch", "moe_dispatch_workspace_size",
-               "router_logits", "router_weight_prepare",
+               "router_logits", "router_weight_prepare", "moe_route_norm_quant_kernels",
                "moe_boundary_supported", "mb_last_error", "mb_device_status"):
         assert fn in names
 
@@ -55,6 +55,13 @@ def test_supported_predicate():
     assert not eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 8200, 256)
     assert not eb.supported(eb.STAGE_ROUTER_LOGITS, 128, 8192, 250)
     assert not eb.supported(99, 8, 16)
+
+
+def test_route_norm_quant_kernels_query_without_device_work():
+    assert eb.route_norm_quant_kernels(0, 8192, 256, 8) == 0
+    assert eb.route_norm_quant_kernels(8192, 8192, 5000, 8) == -1     # E too large
+    assert eb.route_norm_quant_kernels(8192, 8200, 256, 8) == -1      # H not a multiple of 16
+    assert eb.route_norm_quant_kernels(8192, 4096, 256, 8, tp=3) == -1
 
 
 def test_bad_arguments_are_rejected_before_any_launch():

@@ -55,6 +55,38 @@ def test_route_norm_quant_fused(cuda_dev, T, H, E, k, tp):
     assert eb.device_status() == 0
 
 
+@pytest.mark.parametrize("T,H,E,k,tp,gc", [(889, 8192, 256, 8, 1, 0.0), (1500, 2048, 100, 7, 1, 1.0),
+                                           (3001, 4096, 256, 8, 4, 0.0), (2000, 2688, 64, 8, 1, 1.0),
+                                           (1200, 16384, 8, 1, 1, 0.0), (2048, 8192, 256, 32, 1, 1.0),
+                                           (1000, 4096, 512, 8, 1, 0.0), (1300, 1024, 256, 8, 1, 1.0)])
+def test_route_norm_quant_large_batches(cuda_dev, T, H, E, k, tp, gc):
+    """Batches above the beside-router size: the router runs in extra warps of
+    the wide norm-quant kernel (E <= 256, H >= 2048), else before it; either
+    way both outputs equal the oracle's, masked tokens included."""
+    case = synth.make_case("tiny", device=cuda_dev, T=T, H=H, E=E, k=k, tp=tp, gc=gc, join=False)
+    assert (synth.host(case.mask) == 0).any()
+    ids, w, packed, sf = eb.moe_route_norm_quant(case.logits, case.bias, case.mask, case.k, case.x,
+                                                 case.norm_w, case.gc, case.eps, case.gs, tp=tp)
+    torch.cuda.synchronize()
+    ids_o, w_o = oracle.route(synth.host(case.logits), synth.host(case.bias), synth.host(case.mask),
+                              case.k)
+    assert np.array_equal(synth.host(ids), ids_o)
+    assert np.array_equal(synth.host(w).view(np.uint32), w_o.view(np.uint32))
+    p_o, s_o = oracle.norm_quant(synth.host(case.x), case.T, case.H, tp, synth.host(case.norm_w),
+                                 case.gc, case.eps, float(synth.host(case.gs)[0]))
+    assert np.array_equal(synth.host(packed), p_o) and np.array_equal(synth.host(sf), s_o)
+    assert eb.device_status() == 0
+
+
+def test_route_norm_quant_kernel_count(cuda_dev):
+    sms = torch.cuda.get_device_properties(cuda_dev).multi_processor_count
+    assert eb.route_norm_quant_kernels(8192, 8192, 256, 8) == 1
+    assert eb.route_norm_quant_kernels(sms * 6 + 1, 2048, 100, 7) == 1
+    assert eb.route_norm_quant_kernels(sms * 6, 8192, 256, 8) == 2       # router beside the norm-quant
+    assert eb.route_norm_quant_kernels(8192, 8192, 512, 8) == 2          # router first
+    assert eb.route_norm_quant_kernels(8192, 1024, 256, 8) == 2          # not the wide path
+
+
 def test_route_integer_logits_many_ties(cuda_dev):
     g = torch.Generator(device=cuda_dev)
     g.manual_seed(5)
@@ -289,13 +321,14 @@ def test_full_size_sampled(cuda_dev, name):
     assert eb.device_status() == 0
 
 
-@pytest.mark.parametrize("T", [100, 2000])
-def test_joint_pre_expert_steps_feed_the_combine(cuda_dev, T):
+@pytest.mark.parametrize("T,H", [(100, 1024), (2000, 1024), (2000, 2048)])
+def test_joint_pre_expert_steps_feed_the_combine(cuda_dev, T, H):
     """Several steps of (moe_route_norm_quant -> expert_combine) on one stream,
     new logits each step, no synchronisation in between: each step's combine
     must use that step's routing weights (the router running beside the
-    norm-quant at 100 tokens, before it at 2000)."""
-    case = synth.make_case("tiny", device=cuda_dev, T=T, H=1024, E=64, k=8, join=False)
+    norm-quant at 100 tokens, before it at 2000 x 1024, inside it at
+    2000 x 2048)."""
+    case = synth.make_case("tiny", device=cuda_dev, T=T, H=H, E=64, k=8, join=False)
     k, H = case.k, case.H
     ids = torch.empty(T, k, dtype=torch.int32, device=cuda_dev)
     w = torch.empty(T, k, dtype=torch.float32, device=cuda_dev)
@@ -318,4 +351,27 @@ def test_joint_pre_expert_steps_feed_the_combine(cuda_dev, T):
         want = oracle_combine(case, w_o, tokens)
         got = synth.host(out.index_select(0, torch.as_tensor(tokens, device=cuda_dev)))
         assert bf16_ulp_diff(got, want).max() <= 1
+    assert eb.device_status() == 0
+
+
+@pytest.mark.slow
+def test_full_size_joint_sampled(cuda_dev):
+    """The benchmark's pre-expert call at its full size (8192 x 8192, E = 256):
+    router warps inside the norm-quant kernel, sampled tokens against the
+    oracle, masked tokens among them."""
+    case = synth.make_case("prefill", device=cuda_dev)
+    ids, w, packed, sf = eb.moe_route_norm_quant(case.logits, case.bias, case.mask, case.k, case.x,
+                                                 case.norm_w, case.gc, case.eps, case.gs, tp=case.tp)
+    torch.cuda.synchronize()
+    masked = np.nonzero(synth.host(case.mask) == 0)[0][:4]
+    tokens = sample_tokens(case.T, 64, seed=99, must=masked)
+    tk = torch.as_tensor(tokens, device=cuda_dev)
+    ids_o, w_o = oracle.route(synth.host(case.logits.index_select(0, tk)), synth.host(case.bias),
+                              synth.host(case.mask.index_select(0, tk)), case.k)
+    assert np.array_equal(synth.host(ids.index_select(0, tk)), ids_o)
+    assert np.array_equal(synth.host(w.index_select(0, tk)).view(np.uint32), w_o.view(np.uint32))
+    p_o, s_o = oracle.norm_quant(synth.host(case.x_logical().index_select(0, tk)), len(tokens), case.H, 1,
+                                 synth.host(case.norm_w), case.gc, case.eps, float(synth.host(case.gs)[0]))
+    assert np.array_equal(synth.host(packed.index_select(0, tk)), p_o)
+    assert np.array_equal(synth.host(sf.index_select(0, tk)), s_o)
     assert eb.device_status() == 0
