@@ -68,6 +68,7 @@ def _load():
                 "oc_join": (None, [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32]),
                 "oc_dispatch": (None, [P, i32, i32, i32, i32, P, P, P]),
                 "oc_router_logits": (None, [P, i32, i32, P, i32, f32, P, P]),
+                "oc_finalize_allreduce": (None, [P, P, i32, i32, P, P, i32, i32, P, f32, f32, P, P]),
                 "oc_bf16_rn_n": (None, [P, i64, P]),
                 "oc_e4m3_rn_sat_n": (None, [P, i64, P]),
                 "oc_e2m1_code_n": (None, [P, i64, P]),
@@ -233,6 +234,36 @@ def combine(expert_out, R: int, row_idx, wt, w, gc: float, eps: float):
     _load().oc_combine(_ptr(expert_out), int(R), H, _ptr(row_idx), _ptr(wt), T, k, _ptr(w),
                        float(gc), float(eps), _ptr(out))
     return out
+
+
+def finalize_allreduce(expert_outs, Rs, row_idx, wt, w, gc: float, eps: float):
+    """Expert finalize + tensor-parallel all-reduce (TensorRT-LLM PR 21356,
+    "Fused finalize + all-reduce"; PR 21042, MoE paragraph).
+
+    expert_outs: one uint16 [>=R_r, H] array per rank (rows at index >= R_r are
+    never read); Rs: the ranks' row counts; row_idx int32 [world, T, k] (the
+    local row of each slot, -1 where the expert is elsewhere); wt float32 [T, k];
+    w uint16 [H].  Returns (out uint16 [T, H], partials float32 [world, T, H]).
+    """
+    world = len(expert_outs)
+    assert len(Rs) == world
+    eos = [_c(e, np.uint16) for e in expert_outs]
+    H = eos[0].shape[1]
+    assert all(e.shape[1] == H and e.shape[0] >= R for e, R in zip(eos, Rs))
+    row_idx = _c(row_idx, np.int32)
+    assert row_idx.shape[0] == world
+    T, k = row_idx.shape[1], row_idx.shape[2]
+    wt = _c(wt, np.float32)
+    assert wt.shape == (T, k)
+    w = _c(w, np.uint16)
+    ptrs = (ctypes.c_void_p * world)(*[e.ctypes.data for e in eos])
+    rs = np.asarray(Rs, np.int64)
+    out = np.empty((T, H), np.uint16)
+    partials = np.empty((world, T, H), np.float32)
+    _load().oc_finalize_allreduce(ctypes.cast(ptrs, ctypes.c_void_p), _ptr(rs), world, H, _ptr(row_idx),
+                                  _ptr(wt), T, k, _ptr(w), float(gc), float(eps), _ptr(partials),
+                                  _ptr(out))
+    return out, partials
 
 
 def join(residual, branch, gain, alpha: float, beta: float, eps: float,

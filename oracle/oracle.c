@@ -26,6 +26,9 @@
  *  - TensorRT-LLM PR 21356, description, "Router projection": the router
  *    logits come from a projection with FP32 weights and FP32 accumulation,
  *    the BF16 input cast to FP32 and a scale folded in.
+ *  - TensorRT-LLM PR 21356, description, "Fused finalize + all-reduce", and
+ *    PR 21042, MoE paragraph: the expert finalize and the tensor-parallel
+ *    all-reduce of its partials with FP32 accumulation.
  *  - "MoE gate v2" (lmdeploy PR 4835), commit notes: a required token mask;
  *    invalid tokens produce no routing entries; absent rows marked -1; the
  *    gate's routing entries are grouped per expert by a histogram and a scan
@@ -390,6 +393,57 @@ void oc_combine(const uint16_t* expert_out, int64_t R, int H, const int32_t* row
         for (int h = 0; h < H; ++h) out[(size_t)t * H + h] = oc_bf16_rn(acc[h]);
         free(y);
         free(xf);
+        free(acc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Expert finalize fused with the tensor-parallel all-reduce           */
+/* ------------------------------------------------------------------ */
+
+/* TensorRT-LLM PR 21356, description, "Fused finalize + all-reduce" (BF16
+ * TP4 with EP4, the expert finalize and the TP all-reduce in one kernel, FP32
+ * accumulation) and PR 21042, MoE paragraph (the finalize all-reduces
+ * partials in FP32).  Reading: rank r holds the rows of its own experts,
+ * expert_out[r] [R[r], H] BF16, and row_idx[r] [T, k] maps slot j of token t
+ * to a local row, or to -1 / >= R[r] where the slot's expert lives on another
+ * rank (never read).  The routing weights wt [T, k] and the norm weight are
+ * the same on every rank.  Rank r's partial is the combine's FP32
+ * accumulator over its own valid slots in slot order from +0, not rounded;
+ * the all-reduce adds the partials in rank order in FP32 (s = p_0, then
+ * s = s + p_r for r = 1 .. world-1) and every rank outputs bf16(s).
+ * row_idx is [world][T][k]; partial (may be NULL) receives [world][T][H]. */
+void oc_finalize_allreduce(const uint16_t* const* expert_out, const int64_t* R, int world, int H,
+                           const int32_t* row_idx, const float* wt, int T, int k,
+                           const uint16_t* w, float gc, float eps, float* partial,
+                           uint16_t* out) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int t = 0; t < T; ++t) {
+        float* acc = (float*)malloc(sizeof(float) * (size_t)H);
+        float* s = (float*)malloc(sizeof(float) * (size_t)H);
+        float* xf = (float*)malloc(sizeof(float) * (size_t)H);
+        uint16_t* y = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)H);
+        for (int r = 0; r < world; ++r) {
+            for (int h = 0; h < H; ++h) acc[h] = 0.0f;
+            const int32_t* idx = row_idx + ((size_t)r * T + t) * k;
+            for (int j = 0; j < k; ++j) {
+                int64_t row = idx[j];
+                if (row < 0 || row >= R[r]) continue;
+                const uint16_t* src = expert_out[r] + (size_t)row * H;
+                for (int h = 0; h < H; ++h) xf[h] = oc_bf16_to_f32(src[h]);
+                float inv = oc_inv_rms(oc_sumsq(xf, H), H, eps);
+                oc_norm_row(xf, w, gc, inv, H, y);
+                float wj = wt[(size_t)t * k + j];
+                for (int h = 0; h < H; ++h) acc[h] = fmaf(wj, oc_bf16_to_f32(y[h]), acc[h]);
+            }
+            if (partial)
+                memcpy(partial + ((size_t)r * T + t) * H, acc, sizeof(float) * (size_t)H);
+            for (int h = 0; h < H; ++h) s[h] = (r == 0) ? acc[h] : s[h] + acc[h];
+        }
+        for (int h = 0; h < H; ++h) out[(size_t)t * H + h] = oc_bf16_rn(s[h]);
+        free(y);
+        free(xf);
+        free(s);
         free(acc);
     }
 }
