@@ -11,10 +11,13 @@ library cannot be loaded the calls raise.
 from __future__ import annotations
 
 from ._lib import (  # noqa: F401
+    FAR_MAX_WORLD,
+    IPC_HANDLE_BYTES,
     MoEBoundaryError,
     STAGE_COMBINE,
     STAGE_COMBINE_JOIN,
     STAGE_DISPATCH,
+    STAGE_FINALIZE_AR,
     STAGE_JOIN,
     STAGE_NORM_QUANT,
     STAGE_ROUTE,
@@ -24,6 +27,15 @@ from ._lib import (  # noqa: F401
     dispatch_workspace_size,
     expert_combine,
     expert_combine_join,
+    expert_finalize_allreduce,
+    expert_finalize_allreduce_local,
+    finalize_ar_workspace_init,
+    finalize_ar_workspace_size,
+    ipc_alloc,
+    ipc_close,
+    ipc_free,
+    ipc_get_handle,
+    ipc_open,
     last_error,
     lib_path,
     load,

@@ -18,6 +18,9 @@ STAGE_COMBINE_JOIN = 4
 STAGE_ROUTE_NORM_QUANT = 5
 STAGE_DISPATCH = 6
 STAGE_ROUTER_LOGITS = 7
+STAGE_FINALIZE_AR = 8
+FAR_MAX_WORLD = 8
+IPC_HANDLE_BYTES = 64
 
 _lock = threading.Lock()
 _lib = None
@@ -68,6 +71,14 @@ def load() -> ctypes.CDLL:
                 "router_weight_prepare": [P, i32, i32, P, P],
                 "moe_boundary_supported": [i32, i32, i32, i32, i32, i32],
                 "moe_route_norm_quant_kernels": [i32, i32, i32, i32, i32],
+                "finalize_ar_workspace_init": [P, i32, i32, i32, P],
+                "expert_finalize_allreduce": [P, i64, i32, P, P, i32, i32, P, f32, f32, P, i32, i32, i32, P, P],
+                "expert_finalize_allreduce_local": [P, P, i32, P, P, i32, i32, P, f32, f32, P, i32, i32, P, P],
+                "mb_ipc_alloc": [ctypes.c_size_t, P],
+                "mb_ipc_free": [P],
+                "mb_ipc_get_handle": [P, P],
+                "mb_ipc_open": [P, P],
+                "mb_ipc_close": [P],
                 "mb_last_error": [],
                 "mb_device_status": [],
             }
@@ -77,6 +88,8 @@ def load() -> ctypes.CDLL:
                 fn.restype = ctypes.c_char_p if name == "mb_last_error" else ctypes.c_int
             lib.moe_dispatch_workspace_size.argtypes = [i32, i32, i32]
             lib.moe_dispatch_workspace_size.restype = ctypes.c_size_t
+            lib.finalize_ar_workspace_size.argtypes = [i32, i32, i32]
+            lib.finalize_ar_workspace_size.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -403,3 +416,115 @@ def router_logits(x: torch.Tensor, w3: torch.Tensor, scale: float = 1.0,
     _check("router_logits", load().router_logits(_ptr(x), T, H, _ptr(w3), E, float(scale), _ptr(logits),
                                                  _stream(stream)))
     return logits
+
+
+# ---------------------------------------------------------------------------- finalize + all-reduce
+def finalize_ar_workspace_size(world: int, T_max: int, H: int) -> int:
+    """Bytes of one rank's finalize all-reduce workspace (0 when unsupported)."""
+    return int(load().finalize_ar_workspace_size(world, T_max, H))
+
+
+def finalize_ar_workspace_init(workspace, world: int, T_max: int, H: int, stream=None) -> None:
+    """Zero a workspace's call counter and flags (a tensor or a device address)."""
+    ptr = _ptr(workspace) if isinstance(workspace, torch.Tensor) else ctypes.c_void_p(int(workspace))
+    _check("finalize_ar_workspace_init",
+           load().finalize_ar_workspace_init(ptr, world, T_max, H, _stream(stream)))
+
+
+def _addr(x) -> int:
+    return int(x.data_ptr()) if isinstance(x, torch.Tensor) else int(x)
+
+
+def _far_rank_check(fn, expert_out, row_idx, weights, norm_w, out):
+    _want(expert_out, torch.bfloat16, "expert_out")
+    _want(row_idx, torch.int32, "row_idx")
+    _want(weights, torch.float32, "weights")
+    _want(out, torch.bfloat16, "out")
+    H = norm_w.numel()
+    T, k = row_idx.shape
+    if expert_out.dim() != 2 or expert_out.shape[1] != H or weights.shape != (T, k) or out.shape != (T, H):
+        raise ValueError(f"{fn}: shape mismatch")
+
+
+def expert_finalize_allreduce(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
+                              weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
+                              workspaces, rank: int, T_max: int, out: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """One rank's expert finalize + tensor-parallel all-reduce.
+
+    ``workspaces``: every rank's workspace (tensors or device addresses as
+    mapped in this process), in rank order.  Returns out bf16 [T, H], the same
+    on every rank.
+    """
+    _want(norm_w, torch.bfloat16, "norm_w")
+    T, k = row_idx.shape
+    H = norm_w.numel()
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=row_idx.device)
+    _far_rank_check("expert_finalize_allreduce", expert_out, row_idx, weights, norm_w, out)
+    world = len(workspaces)
+    ws = (ctypes.c_void_p * world)(*[_addr(w) for w in workspaces])
+    _check("expert_finalize_allreduce",
+           load().expert_finalize_allreduce(_ptr(expert_out), int(num_rows), H, _ptr(row_idx), _ptr(weights), T, k,
+                                            _ptr(norm_w), float(gain_center), float(eps),
+                                            ctypes.cast(ws, ctypes.c_void_p), world, int(rank), int(T_max),
+                                            _ptr(out), _stream(stream)))
+    return out
+
+
+def expert_finalize_allreduce_local(expert_outs, num_rows, row_idx, weights, norm_w: torch.Tensor,
+                                    gain_center: float, eps: float, workspaces, T_max: int, outs=None,
+                                    stream=None):
+    """All ranks of the exchange in one launch on this device (lists of one
+    entry per rank).  Returns the ranks' outputs (equal to one another)."""
+    _want(norm_w, torch.bfloat16, "norm_w")
+    world = len(expert_outs)
+    if not (len(num_rows) == len(row_idx) == len(weights) == len(workspaces) == world):
+        raise ValueError("expert_finalize_allreduce_local: one entry per rank in every list")
+    T, k = row_idx[0].shape
+    H = norm_w.numel()
+    if outs is None:
+        outs = [torch.empty(T, H, dtype=torch.bfloat16, device=norm_w.device) for _ in range(world)]
+    for r in range(world):
+        if row_idx[r].shape != (T, k):
+            raise ValueError("expert_finalize_allreduce_local: every rank's row_idx must be [T, k]")
+        _far_rank_check("expert_finalize_allreduce_local", expert_outs[r], row_idx[r], weights[r], norm_w, outs[r])
+    arr = lambda xs: (ctypes.c_void_p * world)(*[_addr(x) for x in xs])
+    rows = (ctypes.c_int64 * world)(*[int(n) for n in num_rows])
+    _check("expert_finalize_allreduce_local",
+           load().expert_finalize_allreduce_local(
+               ctypes.cast(arr(expert_outs), ctypes.c_void_p), ctypes.cast(rows, ctypes.c_void_p), H,
+               ctypes.cast(arr(row_idx), ctypes.c_void_p), ctypes.cast(arr(weights), ctypes.c_void_p), T, k,
+               _ptr(norm_w), float(gain_center), float(eps), ctypes.cast(arr(workspaces), ctypes.c_void_p), world,
+               int(T_max), ctypes.cast(arr(outs), ctypes.c_void_p), _stream(stream)))
+    return outs
+
+
+# ---------------------------------------------------------------------------- peer memory (CUDA IPC)
+def ipc_alloc(nbytes: int) -> int:
+    p = ctypes.c_void_p()
+    _check("mb_ipc_alloc", load().mb_ipc_alloc(int(nbytes), ctypes.byref(p)))
+    return int(p.value)
+
+
+def ipc_free(ptr: int) -> None:
+    _check("mb_ipc_free", load().mb_ipc_free(ctypes.c_void_p(int(ptr))))
+
+
+def ipc_get_handle(ptr: int) -> bytes:
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check("mb_ipc_get_handle", load().mb_ipc_get_handle(ctypes.c_void_p(int(ptr)), buf))
+    return buf.raw
+
+
+def ipc_open(handle: bytes) -> int:
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("ipc_open: a handle is 64 bytes")
+    p = ctypes.c_void_p()
+    _check("mb_ipc_open", load().mb_ipc_open(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES),
+                                               ctypes.byref(p)))
+    return int(p.value)
+
+
+def ipc_close(ptr: int) -> None:
+    _check("mb_ipc_close", load().mb_ipc_close(ctypes.c_void_p(int(ptr))))

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_boundary.so")
 SOURCES = ["moe_boundary.cu", "api.cu", "combine.cu", "norm_quant.cu", "route.cu", "decode.cu", "router_proj.cu", "dispatch.cu",
-           "dispatch_noalloc.cu",
+           "dispatch_noalloc.cu", "finalize_ar.cu",
            "common.cuh", "ring.cuh", "route.cuh", "internal.h", "tmap.h"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "moe_boundary.h")
 

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/moe_boundary.h): argument checks, status codes
 // and launches.  No allocation, no synchronisation, no host fallback.
 #include <climits>
+#include <cstring>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -29,6 +30,7 @@ int cuda_status(cudaError_t e, const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
@@ -80,6 +82,11 @@ int moe_boundary_supported(int stage, int T, int H, int E, int k, int tp) {
         case MB_STAGE_DISPATCH:
             return (k >= 1 && k <= kMaxTopK && E >= 1 && E <= kMaxExperts &&
                     static_cast<int64_t>(T) * k <= INT32_MAX)
+                       ? 1
+                       : 0;
+        case MB_STAGE_FINALIZE_AR:
+            return (H >= 16 && H % 16 == 0 && H <= kMaxHidden && k >= 1 && k <= kMaxTopK && tp >= 1 &&
+                    tp <= kFarMaxWorld)
                        ? 1
                        : 0;
         case MB_STAGE_ROUTE_NORM_QUANT:
@@ -293,6 +300,154 @@ int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
     return cuda_status(launch_dispatch(topk_ids, T, k, expert_begin, E, expert_offsets, row_idx, row_token,
                                        workspace, static_cast<cudaStream_t>(stream)),
                        fn);
+}
+
+// ------------------------------------------------------------------ finalize + all-reduce
+static_assert(kFarMaxWorld == MB_FAR_MAX_WORLD, "one limit on the ranks");
+
+static bool far_sizes_ok(int world, int T_max, int H, int k) {
+    return world >= 1 && world <= kFarMaxWorld && T_max >= 1 && H >= 16 && H % 16 == 0 && H <= kMaxHidden &&
+           k >= 1 && k <= kMaxTopK;
+}
+
+size_t finalize_ar_workspace_size(int world, int T_max, int H) {
+    if (!far_sizes_ok(world, T_max, H, 1)) return 0;
+    return finalize_ar_workspace_bytes(world, T_max, H);
+}
+
+int finalize_ar_workspace_init(void* workspace, int world, int T_max, int H, void* stream) {
+    const char* fn = "finalize_ar_workspace_init";
+    if (!far_sizes_ok(world, T_max, H, 1))
+        return fail(MB_ERR_UNSUPPORTED, "%s: needs 1 <= world <= %d, T_max >= 1, H %% 16 == 0, 16 <= H <= %d", fn,
+                    kFarMaxWorld, kMaxHidden);
+    if (!workspace || !aligned256(workspace)) return fail(MB_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", fn);
+    return cuda_status(cudaMemsetAsync(workspace, 0, finalize_ar_flags_bytes(world, T_max),
+                                       static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
+static int check_far_common(const char* fn, int H, int T, int k, int world, int T_max, const uint16_t* norm_w,
+                            void* const* workspaces) {
+    if (T < 0 || H < 0 || k < 0 || world < 0 || T_max < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);
+    if (!far_sizes_ok(world, T_max, H, k))
+        return fail(MB_ERR_UNSUPPORTED,
+                    "%s: needs 1 <= world <= %d, H %% 16 == 0, 16 <= H <= %d, 1 <= k <= %d (world=%d, H=%d, k=%d)", fn,
+                    kFarMaxWorld, kMaxHidden, kMaxTopK, world, H, k);
+    if (T > T_max) return fail(MB_ERR_INVALID_ARG, "%s: T = %d exceeds the workspace's T_max = %d", fn, T, T_max);
+    if (!workspaces || !norm_w) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (!aligned16(norm_w)) return fail(MB_ERR_INVALID_ARG, "%s: norm_w must be 16-byte aligned", fn);
+    for (int q = 0; q < world; ++q)
+        if (!workspaces[q] || !aligned256(workspaces[q]))
+            return fail(MB_ERR_INVALID_ARG, "%s: workspace of rank %d missing or not 256-byte aligned", fn, q);
+    return MB_OK;
+}
+
+static int check_far_rank(const char* fn, int r, const uint16_t* expert_out, int64_t num_rows, const int32_t* row_idx,
+                          const float* weights, const uint16_t* out) {
+    if (num_rows < 0) return fail(MB_ERR_INVALID_ARG, "%s: rank %d: negative num_rows", fn, r);
+    if (!row_idx || !weights || !out || (num_rows > 0 && !expert_out))
+        return fail(MB_ERR_INVALID_ARG, "%s: rank %d: null pointer", fn, r);
+    if (!aligned16(expert_out) || !aligned16(out))
+        return fail(MB_ERR_INVALID_ARG, "%s: rank %d: expert_out and out must be 16-byte aligned", fn, r);
+    return MB_OK;
+}
+
+int expert_finalize_allreduce(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                              const float* weights, int T, int k, const uint16_t* norm_w, float gain_center, float eps,
+                              void* const* workspaces, int world, int rank, int T_max, uint16_t* out, void* stream) {
+    const char* fn = "expert_finalize_allreduce";
+    int st = check_far_common(fn, H, T, k, world, T_max, norm_w, workspaces);
+    if (st != MB_OK) return st;
+    if (rank < 0 || rank >= world) return fail(MB_ERR_INVALID_ARG, "%s: rank %d outside [0, %d)", fn, rank, world);
+    if (T == 0) return MB_OK;
+    st = check_far_rank(fn, rank, expert_out, num_rows, row_idx, weights, out);
+    if (st != MB_OK) return st;
+    FarLaunch L = {};
+    L.nloc = 1;
+    L.expert_out[0] = expert_out;
+    L.R[0] = num_rows;
+    L.row_idx[0] = row_idx;
+    L.wt[0] = weights;
+    L.out[0] = out;
+    for (int q = 0; q < world; ++q) L.ws[q] = workspaces[q];
+    L.w = norm_w;
+    L.gc = gain_center;
+    L.eps = eps;
+    L.H = H;
+    L.T = T;
+    L.k = k;
+    L.Tmax = T_max;
+    L.world = world;
+    L.rank0 = rank;
+    return cuda_status(launch_finalize_ar(L, static_cast<cudaStream_t>(stream)), fn);
+}
+
+int expert_finalize_allreduce_local(const uint16_t* const* expert_out, const int64_t* num_rows, int H,
+                                    const int32_t* const* row_idx, const float* const* weights, int T, int k,
+                                    const uint16_t* norm_w, float gain_center, float eps, void* const* workspaces,
+                                    int world, int T_max, uint16_t* const* out, void* stream) {
+    const char* fn = "expert_finalize_allreduce_local";
+    int st = check_far_common(fn, H, T, k, world, T_max, norm_w, workspaces);
+    if (st != MB_OK) return st;
+    if (T == 0) return MB_OK;
+    if (!expert_out || !num_rows || !row_idx || !weights || !out)
+        return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    FarLaunch L = {};
+    L.nloc = world;
+    for (int r = 0; r < world; ++r) {
+        st = check_far_rank(fn, r, expert_out[r], num_rows[r], row_idx[r], weights[r], out[r]);
+        if (st != MB_OK) return st;
+        L.expert_out[r] = expert_out[r];
+        L.R[r] = num_rows[r];
+        L.row_idx[r] = row_idx[r];
+        L.wt[r] = weights[r];
+        L.out[r] = out[r];
+        L.ws[r] = workspaces[r];
+    }
+    L.w = norm_w;
+    L.gc = gain_center;
+    L.eps = eps;
+    L.H = H;
+    L.T = T;
+    L.k = k;
+    L.Tmax = T_max;
+    L.world = world;
+    L.rank0 = 0;
+    return cuda_status(launch_finalize_ar(L, static_cast<cudaStream_t>(stream)), fn);
+}
+
+// ------------------------------------------------------------------ peer memory
+int mb_ipc_alloc(size_t bytes, void** ptr) {
+    if (!ptr || bytes == 0) return fail(MB_ERR_INVALID_ARG, "mb_ipc_alloc: null pointer or zero size");
+    *ptr = nullptr;
+    return cuda_status(cudaMalloc(ptr, bytes), "mb_ipc_alloc");
+}
+
+int mb_ipc_free(void* ptr) {
+    if (!ptr) return MB_OK;
+    return cuda_status(cudaFree(ptr), "mb_ipc_free");
+}
+
+int mb_ipc_get_handle(const void* ptr, void* handle) {
+    static_assert(sizeof(cudaIpcMemHandle_t) == MB_IPC_HANDLE_BYTES, "IPC handle size");
+    if (!ptr || !handle) return fail(MB_ERR_INVALID_ARG, "mb_ipc_get_handle: null pointer");
+    cudaIpcMemHandle_t h;
+    const int st = cuda_status(cudaIpcGetMemHandle(&h, const_cast<void*>(ptr)), "mb_ipc_get_handle");
+    if (st == MB_OK) std::memcpy(handle, &h, sizeof(h));
+    return st;
+}
+
+int mb_ipc_open(const void* handle, void** ptr) {
+    if (!handle || !ptr) return fail(MB_ERR_INVALID_ARG, "mb_ipc_open: null pointer");
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    return cuda_status(cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess), "mb_ipc_open");
+}
+
+int mb_ipc_close(void* ptr) {
+    if (!ptr) return MB_OK;
+    return cuda_status(cudaIpcCloseMemHandle(ptr), "mb_ipc_close");
 }
 
 int mb_device_status(void) {

@@ -80,4 +80,23 @@ constexpr int kMaxHidden = 16384;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 4096;
 
+// Expert finalize fused with the tensor-parallel all-reduce (finalize_ar.cu).
+constexpr int kFarMaxWorld = 8;
+struct FarLaunch {
+    int nloc;                                   // ranks computed by this launch: rank0 .. rank0 + nloc - 1
+    const uint16_t* expert_out[kFarMaxWorld];   // per local rank
+    int64_t R[kFarMaxWorld];
+    const int32_t* row_idx[kFarMaxWorld];
+    const float* wt[kFarMaxWorld];
+    uint16_t* out[kFarMaxWorld];
+    void* ws[kFarMaxWorld];                     // every rank's workspace, as mapped on this device
+    const uint16_t* w;
+    float gc, eps;
+    int H, T, k, Tmax, world, rank0;
+};
+int far_warps(int H);
+size_t finalize_ar_workspace_bytes(int world, int Tmax, int H);
+size_t finalize_ar_flags_bytes(int world, int Tmax);
+cudaError_t launch_finalize_ar(const FarLaunch& L, cudaStream_t s);
+
 }  // namespace mb

@@ -10,3 +10,4 @@
 #include "router_proj.cu"
 #include "dispatch.cu"
 #include "dispatch_noalloc.cu"
+#include "finalize_ar.cu"

@@ -26,7 +26,7 @@ every masked token carries NaN logits, so a read of either poisons the output.
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional
+from typing import List, Optional
 
 import torch
 
@@ -258,3 +258,55 @@ def host(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return as_u16(t)
     return t.detach().contiguous().cpu().numpy()
+
+
+@dataclasses.dataclass
+class EpCase:
+    """Inputs of the expert finalize + all-reduce with the experts split over
+    `world` ranks (expert e on rank e // (E / world)): per rank, the rows of
+    its own slots (one BF16 N(0, 1) row per slot, in token-major slot order,
+    followed by `nan_tail` NaN rows that must never be read) and its row
+    indices (the local row, -1 for a slot of another rank's expert or of a
+    masked token, and a few slots of other ranks pointing past the end)."""
+    T: int
+    H: int
+    k: int
+    E: int
+    world: int
+    ids: torch.Tensor                 # int32 [T, k] (-1: masked / absent)
+    expert_out: List[torch.Tensor]    # per rank: bfloat16 [R_r + nan_tail, H]
+    R: List[int]
+    row_idx: List[torch.Tensor]       # per rank: int32 [T, k]
+    weights: torch.Tensor             # float32 [T, k] (the same on every rank)
+    norm_w: torch.Tensor              # bfloat16 [H]
+    gc: float
+    eps: float
+
+
+def make_ep_case(T: int, H: int, k: int, E: int, world: int, seed: int, gc: float = 0.0,
+                 masked_frac: float = 0.05, nan_tail: int = 2, device="cpu") -> EpCase:
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    ids = make_topk_ids(T, k, E, seed, masked_frac=masked_frac, invalid_frac=0.01)
+    per = (E + world - 1) // world
+    owner = torch.where(ids >= 0, ids // per, torch.full_like(ids, -1))
+    outs, Rs, idxs = [], [], []
+    for r in range(world):
+        mine = owner == r
+        R = int(mine.sum())
+        idx = torch.full((T, k), -1, dtype=torch.int32)
+        idx[mine] = torch.arange(R, dtype=torch.int32)
+        # some slots of other ranks point past this rank's rows (never read)
+        elsewhere = (owner >= 0) & ~mine & (torch.rand(T, k, generator=gen) < 0.1)
+        idx[elsewhere] = R + torch.randint(0, max(nan_tail, 1), (int(elsewhere.sum()),), generator=gen,
+                                           dtype=torch.int32)
+        rows = torch.empty(R + nan_tail, H, dtype=torch.bfloat16)
+        rows[:R] = torch.randn(R, H, generator=gen).to(torch.bfloat16)
+        rows[R:] = float("nan")
+        outs.append(rows.to(device))
+        Rs.append(R)
+        idxs.append(idx.to(device))
+    weights = torch.rand(T, k, generator=gen).to(device)
+    mean = 1.0 if gc == 0.0 else 0.0
+    norm_w = (mean + 0.1 * torch.randn(H, generator=gen)).to(torch.bfloat16).to(device)
+    return EpCase(T, H, k, E, world, ids.to(device), outs, Rs, idxs, weights, norm_w, gc, 1e-6)

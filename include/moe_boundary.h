@@ -297,6 +297,80 @@ int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
 int moe_dispatch_noalloc(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
                          int32_t* row_idx, int32_t* row_token, void* stream);
 
+/*
+ * Expert finalize fused with the tensor-parallel all-reduce of its partials.
+ *
+ * Source: TensorRT-LLM PR 21356, description, "Fused finalize + all-reduce"
+ * (with the experts split over the ranks, the expert finalize and the TP
+ * all-reduce run as one kernel, a one-shot exchange through peer memory, FP32
+ * accumulation; construction is collective) and PR 21042, MoE paragraph (the
+ * finalize all-reduces partials in FP32).
+ *
+ * Per token t, rank r's partial is the combine's FP32 accumulator over the
+ * slots whose row it holds (0 <= row_idx_r[t, j] < num_rows_r), in slot order
+ * from +0:  acc = fmaf(weights[t, j], bf16((x * (gain_center + norm_w)) *
+ * inv_rms(x)), acc).  Every rank outputs out[t, :] = bf16(((p_0 + p_1) + p_2)
+ * + ...), the partials added in FP32 in rank order.  Slots whose row lives on
+ * another rank are marked -1 (or any value outside [0, num_rows_r)) and never
+ * read.
+ *
+ * Exchange: every rank owns a workspace of finalize_ar_workspace_size()
+ * bytes of device memory that every other rank maps (mb_ipc_* below, or any
+ * other peer mapping); `workspaces` lists all ranks' workspaces as mapped in
+ * the calling process, in rank order.  A call writes this rank's partials
+ * into its own workspace, raises a per-token flag in every rank's workspace,
+ * waits (up to 2 s; then bit 4 of mb_device_status is set and the remaining
+ * tokens are left unwritten) for every rank's flag of each token it reduces,
+ * and reads the peers' partials with plain loads from their memory.  Every
+ * rank must make the same sequence of calls, with the same T, world and T_max;
+ * calls are counted in the workspace (graph replays included), so nothing on
+ * the host changes between calls.  Each launch is cooperative (all CTAs
+ * resident at once).  After a wait ran out the workspaces are out of step:
+ * initialise them again on every rank.
+ *
+ *   expert_out [num_rows, H] BF16    row_idx [T, k] int32   weights [T, k] FP32
+ *   norm_w [H] BF16                  out [T, H] BF16 (out)
+ * Supported: 1 <= world <= 8, H % 16 == 0, 16 <= H <= 16384, 1 <= k <= 32,
+ * T <= T_max.  Pointers 16-byte aligned, workspaces 256-byte aligned.
+ */
+#define MB_FAR_MAX_WORLD 8
+
+/* Bytes of one rank's workspace (0 when the sizes are not supported). */
+size_t finalize_ar_workspace_size(int world, int T_max, int H);
+
+/* Zero a workspace's call counter and flags (enqueued on `stream`); every
+ * rank initialises its own before the first call and after a wait ran out. */
+int finalize_ar_workspace_init(void* workspace, int world, int T_max, int H, void* stream);
+
+/* One rank's call (one process per GPU). */
+int expert_finalize_allreduce(const uint16_t* expert_out, int64_t num_rows, int H, const int32_t* row_idx,
+                              const float* weights, int T, int k, const uint16_t* norm_w, float gain_center, float eps,
+                              void* const* workspaces, int world, int rank, int T_max, uint16_t* out, void* stream);
+
+/* All `world` ranks' calls in one launch on the current device, each rank
+ * with its own inputs, output and workspace (host arrays of `world` entries):
+ * the same exchange and the same results as `world` processes, for tests and
+ * for measuring the kernel on one GPU. */
+int expert_finalize_allreduce_local(const uint16_t* const* expert_out, const int64_t* num_rows, int H,
+                                    const int32_t* const* row_idx, const float* const* weights, int T, int k,
+                                    const uint16_t* norm_w, float gain_center, float eps, void* const* workspaces,
+                                    int world, int T_max, uint16_t* const* out, void* stream);
+
+/*
+ * Peer memory through CUDA IPC (one process per GPU, one node).
+ * mb_ipc_alloc: a whole cudaMalloc allocation (its handle maps from its
+ * first byte).  mb_ipc_get_handle: the MB_IPC_HANDLE_BYTES-byte handle of such
+ * an allocation, to send to the peers.  mb_ipc_open: map a peer's handle in
+ * this process.  mb_ipc_close: unmap it.  A rank frees its own allocation only
+ * after every peer has closed its mapping of it.
+ */
+#define MB_IPC_HANDLE_BYTES 64
+int mb_ipc_alloc(size_t bytes, void** ptr);
+int mb_ipc_free(void* ptr);
+int mb_ipc_get_handle(const void* ptr, void* handle);
+int mb_ipc_open(const void* handle, void** ptr);
+int mb_ipc_close(void* ptr);
+
 /* Stage ids for moe_boundary_supported(). */
 enum {
     MB_STAGE_ROUTE = 0,
@@ -307,6 +381,7 @@ enum {
     MB_STAGE_ROUTE_NORM_QUANT = 5,
     MB_STAGE_DISPATCH = 6,
     MB_STAGE_ROUTER_LOGITS = 7,
+    MB_STAGE_FINALIZE_AR = 8,   /* tp = world */
 };
 
 /*
@@ -324,7 +399,8 @@ const char* mb_last_error(void);
  * current device (synchronous).  Bit 0: a producer's bounded wait for a free
  * shared-memory slot ran out; bit 1: a drain wait ran out; bit 2: a
  * consumer's wait for a copied row ran out; bit 3: the router projection's
- * wait for its tensor-core MMAs ran out.  0 means no kernel reported a
+ * wait for its tensor-core MMAs ran out; bit 4: the finalize all-reduce's
+ * wait for a peer's partial ran out.  0 means no kernel reported a
  * timeout since the last call.  Returns -1 (and sets mb_last_error) when the
  * CUDA runtime fails.
  */

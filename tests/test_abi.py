@@ -130,3 +130,13 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         eb.norm_quant_nvfp4(x, 4, torch.zeros(64, dtype=torch.bfloat16), 0.0, 1e-6,
                             torch.ones(1))
+
+
+def test_finalize_ar_sizes_without_device_work():
+    assert eb.finalize_ar_workspace_size(4, 128, 8192) > 4 * 128 * 8192 * 2
+    assert eb.finalize_ar_workspace_size(9, 128, 8192) == 0      # more ranks than the kernel takes
+    assert eb.finalize_ar_workspace_size(4, 128, 8200) == 0      # H not a multiple of 16
+    assert eb.finalize_ar_workspace_size(4, 0, 8192) == 0
+    assert eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 8, 4)
+    assert not eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 8, 9)
+    assert not eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 33, 4)
