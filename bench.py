@@ -314,6 +314,7 @@ def run_ours(args, info):
 
     disp = None if args.no_dispatch else run_dispatch(eb, ids, E, dev, reps=max(5, min(args.steps, 200)))
     dec = None if args.no_decode else run_decode(eb, dev, reps=max(5, min(args.steps, 100)))
+    far = None if args.no_finalize_ar else run_finalize_ar(eb, dev, peak, reps=max(5, min(args.steps, 100)))
 
     # end to end through the same calls with host buffers (pinned), copies inside
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
@@ -357,6 +358,7 @@ def run_ours(args, info):
             "e2e": e2e,
             "dispatch": disp,
             "decode": dec,
+            "finalize_allreduce": far,
             "gpu_launches": (pre_kernels + 1) * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
@@ -466,6 +468,37 @@ def run_decode(eb, dev, reps):
     return r
 
 
+def run_finalize_ar(eb, dev, peak, reps):
+    """The expert finalize fused with the tensor-parallel all-reduce at the
+    pages' decode size (128 tokens of width 8192, top-8 of 256 experts split
+    over 4 ranks), all four ranks' kernels in one launch on this GPU, each
+    with its own workspace: on one device the peers' partials are read from
+    local HBM, so the number measures the kernel, not NVLink."""
+    from expert_combine_b200 import synth
+    world, T, H, k, E = 4, 128, 8192, 8, 256
+    c = synth.make_ep_case(T, H, k, E, world, seed=synth.SEEDS["decode"] + 11, device=dev)
+    n = eb.finalize_ar_workspace_size(world, T, H)
+    ws = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(world)]
+    for w in ws:
+        eb.finalize_ar_workspace_init(w, world, T, H)
+    outs = [torch.empty(T, H, dtype=torch.bfloat16, device=dev) for _ in range(world)]
+
+    def call():
+        eb.expert_finalize_allreduce_local(c.expert_out, c.R, c.row_idx, [c.weights] * world, c.norm_w, c.gc,
+                                           c.eps, ws, T, outs=outs)
+
+    us = _graph_us(call, reps, dev)
+    rows = sum(c.R)
+    # bytes of the one launch: every rank reads its rows, writes its partial,
+    # reads all ranks' partials, writes its output; indices and weights
+    hbm = rows * 2 * H + world * (T * H * 4 + world * T * H * 4 + T * H * 2 + T * k * 8)
+    gbs = hbm / (us * 1e-6) / 1e9
+    return {"workload": f"T={T} H={H} E={E} k={k}, experts split over {world} ranks, one-device exchange",
+            "us": us, "bytes": hbm, "gbs": gbs, "frac_of_measured_hbm": gbs / peak, "bound": "hbm",
+            "nvlink_bytes_per_rank": (world - 1) * T * H * 4,
+            "how": f"{reps} calls per CUDA graph, one replay between two events"}
+
+
 def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, pre_expert, steps):
     """Host inputs (pinned) -> device -> the three calls -> host outputs, per step."""
     T, H, k = case.T, case.H, case.k
@@ -513,6 +546,8 @@ def main():
     ap.add_argument("--no-dispatch", action="store_true",
                     help="skip the separate timing of the dispatch step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-finalize-ar", action="store_true",
+                    help="skip the separate timing of the finalize + all-reduce (one-device exchange)")
     ap.add_argument("--separate", action="store_true",
                     help="issue moe_route and norm_quant_nvfp4 as two calls instead of moe_route_norm_quant")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

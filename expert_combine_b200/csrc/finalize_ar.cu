@@ -69,12 +69,26 @@ struct FarArgs {
 
 constexpr unsigned int kFarWaitCode = 16u;   // mb_device_status bit 4
 
-__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Release / acquire as fence + relaxed access: a thread's fence orders every
+// write it has observed (the CTA's, through the barrier before it) before its
+// later flag stores, and its flag loads before every later read of the CTA
+// (through the barrier after it).  SYS: some ranks are other processes'
+// GPUs (system scope); otherwise every rank is on this device (GPU scope).
+template <bool SYS>
+__device__ __forceinline__ void fence_scope() {
+    if constexpr (SYS) asm volatile("fence.acq_rel.sys;" ::: "memory");
+    else asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
-__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+template <bool SYS>
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+    if constexpr (SYS) asm volatile("st.relaxed.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    else asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+template <bool SYS>
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
     uint32_t v;
-    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if constexpr (SYS) asm volatile("ld.relaxed.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    else asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 // A peer's partial: cached in L2 only (the line may have changed since an
@@ -131,7 +145,7 @@ __device__ __forceinline__ float2 far_norm_pair(uint32_t xw, uint32_t wpw, float
 
 // One CTA of NW warps per (token group, rank); thread tid owns elements
 // [32 tid, 32 tid + 32).
-template <int NW, bool GC0>
+template <int NW, bool GC0, bool SYS>
 __global__ void __launch_bounds__(NW * 32) finalize_ar_kernel(const FarArgs a) {
     __shared__ float red[2 * NW];
     __shared__ int s_abort;
@@ -219,67 +233,69 @@ __global__ void __launch_bounds__(NW * 32) finalize_ar_kernel(const FarArgs a) {
             if (c / 4 < nvalid)
                 *reinterpret_cast<float4*>(prow + 4 * c) =
                     make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y);
-        __syncthreads();
-        if (tid == 0) {   // the partial of t is in memory: tell every rank
-            __threadfence_system();
-            for (int q = 0; q < world; ++q) {
-                uint32_t* f = reinterpret_cast<uint32_t*>(a.ws[q] + foff) + static_cast<size_t>(rank) * a.Tmax + t;
-                st_release_sys(f, epoch);
-            }
-        }
     }
 
-    // ---- phase 2: every rank's partial of the CTA's tokens, summed in rank order
-    const uint32_t* my_flags = reinterpret_cast<const uint32_t*>(my_ws + foff);
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        if (tid == 0) {
-            const unsigned long long t0 = globaltimer_ns();
-            bool ok = true;
-            for (int q = 0; q < world && ok; ++q) {
-                const uint32_t* f = my_flags + static_cast<size_t>(q) * a.Tmax + t;
-                while (ld_acquire_sys(f) != epoch) {
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                        atomicOr(&g_wait_timeout, kFarWaitCode);
-                        ok = false;
-                        break;
+    // ---- the CTA's partials are in memory: thread q tells rank q (one
+    // system-scope fence per thread, then plain flag stores), then waits for
+    // rank q's flags of the CTA's tokens (plain loads, one fence after them)
+    __syncthreads();
+    if (tid < world) {
+        fence_scope<SYS>();
+        uint32_t* f = reinterpret_cast<uint32_t*>(a.ws[tid] + foff) + static_cast<size_t>(rank) * a.Tmax;
+        for (int t = blockIdx.x; t < T; t += gridDim.x) st_relaxed<SYS>(f + t, epoch);
+        const uint32_t* mine = reinterpret_cast<const uint32_t*>(my_ws + foff) + static_cast<size_t>(tid) * a.Tmax;
+        const unsigned long long t0 = globaltimer_ns();
+        bool ok = true;
+        for (int t = blockIdx.x; t < T && ok; t += gridDim.x) {
+            while (ld_relaxed<SYS>(mine + t) != epoch) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(&g_wait_timeout, kFarWaitCode);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        fence_scope<SYS>();
+        if (!ok) s_abort = 1;
+    }
+    __syncthreads();
+
+    // ---- phase 2: every rank's partial of the CTA's tokens, summed in rank
+    // order; here thread tid takes the float4 columns tid, tid + 32 NW, ...
+    // (every warp access one contiguous run)
+    const int ncol = H / 4;
+    for (int t = blockIdx.x; t < T && s_abort == 0; t += gridDim.x) {
+        uint16_t* orow = io.out + static_cast<size_t>(t) * H;
+        for (int c0 = tid; c0 < ncol; c0 += 4 * NW * 32) {
+            float4 sum[4];
+#pragma unroll
+            for (int q = 0; q < kFarMaxWorld; ++q) {
+                if (q >= world) break;
+                const float4* src = reinterpret_cast<const float4*>(a.ws[q] + poff) + static_cast<size_t>(t) * ncol;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * NW * 32;
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (c < ncol) v = ld_cg_f4(reinterpret_cast<const float*>(src + c));
+                    if (q == 0) {
+                        sum[u] = v;
+                    } else {
+                        sum[u].x = __fadd_rn(sum[u].x, v.x);
+                        sum[u].y = __fadd_rn(sum[u].y, v.y);
+                        sum[u].z = __fadd_rn(sum[u].z, v.z);
+                        sum[u].w = __fadd_rn(sum[u].w, v.w);
                     }
                 }
             }
-            if (!ok) s_abort = 1;
-        }
-        __syncthreads();
-        if (s_abort != 0) break;
-        float s[32];
 #pragma unroll
-        for (int q = 0; q < kFarMaxWorld; ++q) {
-            if (q >= world) break;
-            const float* src = reinterpret_cast<const float*>(a.ws[q] + poff) + static_cast<size_t>(t) * H + 32 * tid;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (c / 4 < nvalid) v = ld_cg_f4(src + 4 * c);
-                if (q == 0) {
-                    s[4 * c] = v.x;
-                    s[4 * c + 1] = v.y;
-                    s[4 * c + 2] = v.z;
-                    s[4 * c + 3] = v.w;
-                } else {
-                    s[4 * c] = __fadd_rn(s[4 * c], v.x);
-                    s[4 * c + 1] = __fadd_rn(s[4 * c + 1], v.y);
-                    s[4 * c + 2] = __fadd_rn(s[4 * c + 2], v.z);
-                    s[4 * c + 3] = __fadd_rn(s[4 * c + 3], v.w);
-                }
+            for (int u = 0; u < 4; ++u) {
+                const int c = c0 + u * NW * 32;
+                if (c < ncol)
+                    *reinterpret_cast<uint2*>(orow + 4 * c) =
+                        make_uint2(pack_bf16x2_rn(make_float2(sum[u].x, sum[u].y)),
+                                   pack_bf16x2_rn(make_float2(sum[u].z, sum[u].w)));
             }
         }
-        uint16_t* orow = io.out + static_cast<size_t>(t) * H + 32 * tid;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            if (c / 2 < nvalid)
-                *reinterpret_cast<uint4*>(orow + 8 * c) =
-                    make_uint4(pack_bf16x2_rn(make_float2(s[8 * c], s[8 * c + 1])),
-                               pack_bf16x2_rn(make_float2(s[8 * c + 2], s[8 * c + 3])),
-                               pack_bf16x2_rn(make_float2(s[8 * c + 4], s[8 * c + 5])),
-                               pack_bf16x2_rn(make_float2(s[8 * c + 6], s[8 * c + 7])));
     }
 
     // ---- the last CTA of this rank to finish publishes the epoch for the next call
@@ -295,9 +311,9 @@ __global__ void __launch_bounds__(NW * 32) finalize_ar_kernel(const FarArgs a) {
     }
 }
 
-template <int NW, bool GC0>
+template <int NW, bool GC0, bool SYS>
 cudaError_t launch_far_nw(const FarArgs& a, int nloc, cudaStream_t s) {
-    auto kern = finalize_ar_kernel<NW, GC0>;
+    auto kern = finalize_ar_kernel<NW, GC0, SYS>;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NW * 32, 0);
     if (e != cudaSuccess) return e;
@@ -316,14 +332,14 @@ cudaError_t launch_far_nw(const FarArgs& a, int nloc, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <bool GC0>
+template <bool GC0, bool SYS>
 cudaError_t launch_far_gc(const FarArgs& a, int nloc, cudaStream_t s) {
     switch (far_warps(a.H)) {
-        case 1: return launch_far_nw<1, GC0>(a, nloc, s);
-        case 2: return launch_far_nw<2, GC0>(a, nloc, s);
-        case 4: return launch_far_nw<4, GC0>(a, nloc, s);
-        case 8: return launch_far_nw<8, GC0>(a, nloc, s);
-        case 16: return launch_far_nw<16, GC0>(a, nloc, s);
+        case 1: return launch_far_nw<1, GC0, SYS>(a, nloc, s);
+        case 2: return launch_far_nw<2, GC0, SYS>(a, nloc, s);
+        case 4: return launch_far_nw<4, GC0, SYS>(a, nloc, s);
+        case 8: return launch_far_nw<8, GC0, SYS>(a, nloc, s);
+        case 16: return launch_far_nw<16, GC0, SYS>(a, nloc, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -358,7 +374,10 @@ cudaError_t launch_finalize_ar(const FarLaunch& L, cudaStream_t s) {
     a.Tmax = L.Tmax;
     a.world = L.world;
     a.rank0 = L.rank0;
-    return L.gc == 0.0f ? launch_far_gc<true>(a, L.nloc, s) : launch_far_gc<false>(a, L.nloc, s);
+    // every rank on this device: GPU-scope ordering suffices; else system scope
+    if (L.nloc == L.world)
+        return L.gc == 0.0f ? launch_far_gc<true, false>(a, L.nloc, s) : launch_far_gc<false, false>(a, L.nloc, s);
+    return L.gc == 0.0f ? launch_far_gc<true, true>(a, L.nloc, s) : launch_far_gc<false, true>(a, L.nloc, s);
 }
 
 }  // namespace mb
