@@ -13,8 +13,10 @@
 // into a 32-bit order-preserving key; k merge rounds then emit the picks in
 // order, each a warp max (redux.sync) over the lanes' current bests with the
 // lowest expert id winning among equal keys (a warp min over the tied
-// lanes).  For E <= 512 a lane rescans its own <= 16 scores after a pick;
-// beyond that it keeps a sorted list of its best k.  Nothing is staged in
+// lanes).  For E <= 512 a lane keeps its best and second-best remaining
+// scores, promotes the second when its best is picked and rescans its <= 16
+// scores only when picked again before a rescan; beyond that it keeps a
+// sorted list of its best k.  Nothing is staged in
 // shared or global scratch memory.
 #include "internal.h"
 #include "route.cuh"

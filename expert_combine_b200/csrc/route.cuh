@@ -88,8 +88,66 @@ __device__ __forceinline__ void load_logits(const float* l, int E, int lane, boo
     }
 }
 
-// E <= 32 * EPL: every lane keeps its EPL scores and rescans them after each
-// of its picks.
+// Expert id of position p of this lane's scores (4 per 128-bit load,
+// ids 4 * (lane + 32 u) + i for position 4 u + i).
+__device__ __forceinline__ uint32_t lane_pos_id(int p, int lane) {
+    return 4u * static_cast<uint32_t>(lane + 32 * (p >> 2)) + static_cast<uint32_t>(p & 3);
+}
+
+// A lane's remaining candidates for the merge rounds: its best and
+// second-best keys not yet picked (largest key, lowest position -- hence
+// lowest id -- among equals) and the positions already picked.  When its
+// best is picked the second is promoted; only a lane picked twice in a row
+// without a rescan in between scans its scores again, so most rounds cost a
+// few instructions instead of a rescan.
+template <int EPL>
+struct LaneTop2 {
+    uint32_t k1, k2, id1, id2;
+    int p1, p2;
+    uint32_t used;
+    bool have2;
+
+    __device__ __forceinline__ void scan(const uint32_t (&key)[EPL], int lane) {
+        k1 = k2 = 0u;
+        p1 = p2 = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const uint32_t v = ((used >> i) & 1u) ? 0u : key[i];
+            if (v > k1) {
+                k2 = k1;
+                p2 = p1;
+                k1 = v;
+                p1 = i;
+            } else if (v > k2) {
+                k2 = v;
+                p2 = i;
+            }
+        }
+        id1 = lane_pos_id(p1, lane);
+        id2 = lane_pos_id(p2, lane);
+        have2 = true;
+    }
+    __device__ __forceinline__ void init(const uint32_t (&key)[EPL], int lane) {
+        used = 0u;
+        scan(key, lane);
+    }
+    // this lane's best was picked
+    __device__ __forceinline__ void pop(const uint32_t (&key)[EPL], int lane) {
+        used |= 1u << p1;
+        if (have2) {
+            k1 = k2;
+            p1 = p2;
+            id1 = id2;
+            have2 = false;
+        } else {
+            scan(key, lane);
+        }
+    }
+};
+
+// E <= 32 * EPL: every lane keeps its EPL scores; k merge rounds, each a warp
+// max over the lanes' best remaining keys, the lowest id among the lanes
+// holding it winning.
 template <int EPL>
 __device__ __forceinline__ void select_small(const float (&lv)[EPL], const float* bias, int E, int k, int lane,
                                              bool vec, uint32_t& pick_key, uint32_t& pick_id) {
@@ -111,29 +169,11 @@ __device__ __forceinline__ void select_small(const float (&lv)[EPL], const float
             }
         }
     }
-    // lane best: the largest key, lowest position among equals
-    auto best_of = [&](uint32_t& bk, int& bp) {
-        bk = 0u;
-        bp = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i)
-            if (key[i] > bk) {
-                bk = key[i];
-                bp = i;
-            }
-    };
-    uint32_t bk;
-    int bp;
-    best_of(bk, bp);
+    LaneTop2<EPL> c;
+    c.init(key, lane);
     for (int j = 0; j < k; ++j) {
-        const uint32_t my_id = 4u * static_cast<uint32_t>(lane + 32 * (bp >> 2)) + static_cast<uint32_t>(bp & 3);
         uint32_t key_j, id_j;
-        if (pick_round(bk, my_id, key_j, id_j)) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == bp) key[i] = 0u;
-            best_of(bk, bp);
-        }
+        if (pick_round(c.k1, c.id1, key_j, id_j)) c.pop(key, lane);
         if (lane == j) {
             pick_key = key_j;
             pick_id = id_j;
@@ -169,39 +209,16 @@ __device__ __forceinline__ void select_small2(const float (&la)[EPL], const floa
             kb[4 * u + i] = (vb && in) ? score_key(__fadd_rn(sigmoid_fixed(lb[4 * u + i]), bb[i])) : 0u;
         }
     }
-    auto best_of = [&](const uint32_t (&key)[EPL], uint32_t& bk, int& bp) {
-        bk = 0u;
-        bp = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i)
-            if (key[i] > bk) {
-                bk = key[i];
-                bp = i;
-            }
-    };
-    uint32_t bka, bkb;
-    int bpa, bpb;
-    best_of(ka, bka, bpa);
-    best_of(kb, bkb, bpb);
+    LaneTop2<EPL> ca, cb;
+    ca.init(ka, lane);
+    cb.init(kb, lane);
     for (int j = 0; j < k; ++j) {
-        const uint32_t ida = 4u * static_cast<uint32_t>(lane + 32 * (bpa >> 2)) + static_cast<uint32_t>(bpa & 3);
-        const uint32_t idb = 4u * static_cast<uint32_t>(lane + 32 * (bpb >> 2)) + static_cast<uint32_t>(bpb & 3);
-        const uint32_t ma = warp_max_u32(bka);
-        const uint32_t mb = warp_max_u32(bkb);
-        const uint32_t wa = warp_min_u32(bka == ma ? ida : 0xffffffffu);
-        const uint32_t wb = warp_min_u32(bkb == mb ? idb : 0xffffffffu);
-        if (bka == ma && ida == wa) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == bpa) ka[i] = 0u;
-            best_of(ka, bka, bpa);
-        }
-        if (bkb == mb && idb == wb) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i)
-                if (i == bpb) kb[i] = 0u;
-            best_of(kb, bkb, bpb);
-        }
+        const uint32_t ma = warp_max_u32(ca.k1);
+        const uint32_t mb = warp_max_u32(cb.k1);
+        const uint32_t wa = warp_min_u32(ca.k1 == ma ? ca.id1 : 0xffffffffu);
+        const uint32_t wb = warp_min_u32(cb.k1 == mb ? cb.id1 : 0xffffffffu);
+        if (ca.k1 == ma && ca.id1 == wa) ca.pop(ka, lane);
+        if (cb.k1 == mb && cb.id1 == wb) cb.pop(kb, lane);
         if (lane == j) {
             pick_a = wa;
             pick_b = wb;
