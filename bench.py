@@ -381,7 +381,8 @@ def run_dispatch(eb, ids, E, dev, reps):
     ws = torch.empty(max(1, eb.dispatch_workspace_size(T, k, E)), dtype=torch.uint8, device=dev)
     us = _graph_us(lambda: eb.moe_dispatch(ids, E, 0, off, idx, tok, ws), reps, dev)
     n = T * k
-    kernels = 1 if eb.dispatch_workspace_size(T, k, E) == 0 else 3
+    tiles = (n + 4095) // 4096    # 4096 entries per tile; the column scan runs above 32 tiles
+    kernels = 1 if tiles <= 1 else (2 if tiles <= 32 else 3)
     return {"us": us, "entries": n, "experts": E, "kernels": kernels,
             "bytes": 12 * n, "gbs": 12 * n / (us * 1e-6) / 1e9,
             "bound": "latency", "how": f"{reps} calls per CUDA graph, one replay between two events",

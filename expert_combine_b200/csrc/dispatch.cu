@@ -21,9 +21,10 @@
 // lanes in its group: the order of i is kept without sorting.  Per-warp counts are then scanned across the
 // eight warps of the tile (shared memory), across tiles per expert, and over
 // experts.  One tile (T * k <= 4096, decode batches) runs as one kernel;
-// larger inputs run three kernels: tile counts, the column scan over tiles
-// (one CTA per 32 experts) and the placement, with the per-tile counts in the
-// caller's workspace.  Everything is integer, so the result is exact and
+// larger inputs run the tile counts and the placement, with the per-tile
+// counts in the caller's workspace; above 32 tiles a column scan over the
+// tiles (one CTA per 32 experts) runs between them, below it each placement
+// CTA sums the counts of the tiles before its own.  Everything is integer, so the result is exact and
 // independent of the launch shape.
 #include <mutex>
 
@@ -39,6 +40,7 @@ constexpr int kDispThreads = kDispWarps * 32;
 constexpr int kDispIter = 16;                                  // 32-entry steps per warp
 constexpr int kDispWarpSpan = 32 * kDispIter;                  // 512 entries per warp
 constexpr int kDispTile = kDispWarps * kDispWarpSpan;          // 4096 entries per CTA
+constexpr int kDispFoldTiles = 32;   // up to this many tiles the placement scans the tile counts itself
 
 struct DispatchArgs {
     const int32_t* ids;
@@ -296,6 +298,10 @@ __global__ void __launch_bounds__(kScanWarps * 32) dispatch_scan_kernel(const Di
 
 // Kernel 3: offsets from the totals (every CTA scans them; CTA 0 writes them
 // out), then each entry's row = offsets[e] + tile base of e + rank in tile.
+// FOLD (few tiles): kernel 2 is skipped and every CTA forms its own tile
+// bases and the totals from the raw per-tile counts (ntiles * E loads per
+// CTA, all of them L2 hits).
+template <bool FOLD>
 __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(const DispatchArgs a) {
     extern __shared__ __align__(16) int32_t dsm[];
     int32_t* add = dsm;          // [E]
@@ -306,13 +312,31 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(const Disp
     load_tile4<false>(a.row_idx, a.n, -1, v);   // packed (expert, rank) from kernel 1; rewritten below
     // this tile's bases per expert, fetched beside the totals (E <= 16 * 256)
     constexpr int kPer = kMaxExperts / kDispThreads;
-    const int32_t* tb = a.tile_counts + static_cast<int64_t>(blockIdx.x) * a.E;
     int base[kPer];
+    if constexpr (FOLD) {
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int e = threadIdx.x + j * kDispThreads;
-        base[j] = e < a.E ? __ldg(tb + e) : 0;
-        if (e < a.E) add[e] = __ldg(a.totals + e);
+        for (int j = 0; j < kPer; ++j) {
+            const int e = threadIdx.x + j * kDispThreads;
+            int sum = 0, mine = 0;
+            if (e < a.E) {
+#pragma unroll 8
+                for (int t = 0; t < a.ntiles; ++t) {
+                    const int c = __ldg(a.tile_counts + static_cast<int64_t>(t) * a.E + e);
+                    mine = (t == static_cast<int>(blockIdx.x)) ? sum : mine;
+                    sum += c;
+                }
+                add[e] = sum;
+            }
+            base[j] = mine;
+        }
+    } else {
+        const int32_t* tb = a.tile_counts + static_cast<int64_t>(blockIdx.x) * a.E;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int e = threadIdx.x + j * kDispThreads;
+            base[j] = e < a.E ? __ldg(tb + e) : 0;
+            if (e < a.E) add[e] = __ldg(a.totals + e);
+        }
     }
     __syncthreads();
     const int R = block_exclusive_scan(add, a.E, ws);
@@ -407,12 +431,13 @@ cudaError_t launch_dispatch(const int32_t* ids, int T, int k, int e0, int E, int
     cudaLaunchConfig_t c1 = pdl_config(static_cast<int>(nt), kDispThreads, smem1, s, attr);
     err = cudaLaunchKernelEx(&c1, dispatch_count_kernel, a);
     if (err != cudaSuccess) return err;
+    const size_t smem3 = (static_cast<size_t>(E) + kDispWarps) * sizeof(int32_t);
+    cudaLaunchConfig_t c3 = pdl_config(static_cast<int>(nt), kDispThreads, smem3, s, attr);
+    if (nt <= kDispFoldTiles) return cudaLaunchKernelEx(&c3, dispatch_place_kernel<true>, a);
     cudaLaunchConfig_t c2 = pdl_config((E + 31) / 32, kScanWarps * 32, 0, s, attr);
     err = cudaLaunchKernelEx(&c2, dispatch_scan_kernel, a);
     if (err != cudaSuccess) return err;
-    const size_t smem3 = (static_cast<size_t>(E) + kDispWarps) * sizeof(int32_t);
-    cudaLaunchConfig_t c3 = pdl_config(static_cast<int>(nt), kDispThreads, smem3, s, attr);
-    return cudaLaunchKernelEx(&c3, dispatch_place_kernel, a);
+    return cudaLaunchKernelEx(&c3, dispatch_place_kernel<false>, a);
 }
 
 }  // namespace mb
