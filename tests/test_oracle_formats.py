@@ -8,7 +8,6 @@ in float64, or hand-derived binary32 results.
 import os
 
 import numpy as np
-import pytest
 import torch
 
 import oracle
