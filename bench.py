@@ -591,6 +591,8 @@ def main():
                     help="issue moe_route and norm_quant_nvfp4 as two calls instead of moe_route_norm_quant")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="NVTX ranges around every library call (for a profiler's timeline)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -599,7 +601,11 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, info)
-        run_ours(args, info)
+        import contextlib
+
+        import expert_combine_b200 as eb
+        with eb.trace() if args.nvtx else contextlib.nullcontext():
+            run_ours(args, info)
         return 0
     finally:
         if args.impl == "ours":

@@ -49,4 +49,6 @@ from ._lib import (  # noqa: F401
     router_logits,
     router_weight_prepare,
     supported,
+    trace,
+    tracing,
 )

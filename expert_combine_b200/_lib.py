@@ -10,6 +10,50 @@ import torch
 
 from . import build as _build
 
+# ---------------------------------------------------------------------------- NVTX ranges
+# Off by default (no cost beyond one flag test per call).  Inside `trace()`,
+# every call of the binding is an NVTX range named after its C entry point,
+# so a profiler's timeline (or `ncu --nvtx --nvtx-include`) can pick out the
+# boundary's kernels by call.
+_trace_depth = 0
+
+
+class trace:
+    """Context manager: NVTX ranges around every call of the library while active."""
+
+    def __enter__(self):
+        global _trace_depth
+        _trace_depth += 1
+        return self
+
+    def __exit__(self, *exc):
+        global _trace_depth
+        _trace_depth -= 1
+        return False
+
+
+def tracing() -> bool:
+    return _trace_depth > 0
+
+
+def _traced(fn):
+    name = fn.__name__
+
+    def wrapper(*args, **kwargs):
+        if _trace_depth <= 0:
+            return fn(*args, **kwargs)
+        torch.cuda.nvtx.range_push(name)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    wrapper.__name__ = name
+    wrapper.__qualname__ = fn.__qualname__
+    wrapper.__doc__ = fn.__doc__
+    wrapper.__wrapped__ = fn
+    return wrapper
+
 STAGE_ROUTE = 0
 STAGE_NORM_QUANT = 1
 STAGE_COMBINE = 2
@@ -134,6 +178,7 @@ def device_status() -> int:
     return v
 
 
+@_traced
 def moe_route(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor, k: int,
               topk_ids: Optional[torch.Tensor] = None, topk_weights: Optional[torch.Tensor] = None,
               stream=None):
@@ -156,6 +201,7 @@ def moe_route(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor
     return topk_ids, topk_weights
 
 
+@_traced
 def norm_quant_nvfp4(x: torch.Tensor, num_tokens: int, norm_w: torch.Tensor, gain_center: float,
                      eps: float, global_scale: torch.Tensor, tp: int = 1,
                      packed: Optional[torch.Tensor] = None, sf: Optional[torch.Tensor] = None,
@@ -186,6 +232,7 @@ def norm_quant_nvfp4(x: torch.Tensor, num_tokens: int, norm_w: torch.Tensor, gai
     return packed, sf
 
 
+@_traced
 def moe_route_norm_quant(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor, k: int,
                          x: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
                          global_scale: torch.Tensor, tp: int = 1,
@@ -233,6 +280,7 @@ def route_norm_quant_kernels(M: int, H: int, E: int, k: int, tp: int = 1) -> int
     device (for a 16-byte-aligned x); -1 when unsupported or without a device."""
     return int(load().moe_route_norm_quant_kernels(M, H, tp, E, k))
 
+@_traced
 def expert_combine(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
                    weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
                    out: Optional[torch.Tensor] = None, stream=None):
@@ -255,6 +303,7 @@ def expert_combine(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tenso
     return out
 
 
+@_traced
 def residual_join(residual: torch.Tensor, branch: torch.Tensor, gain: torch.Tensor, alpha: float,
                   beta: float, eps: float, next_w: Optional[torch.Tensor] = None,
                   next_gc: float = 1.0, next_eps: float = 1e-6,
@@ -278,6 +327,7 @@ def residual_join(residual: torch.Tensor, branch: torch.Tensor, gain: torch.Tens
     return next_prenorm
 
 
+@_traced
 def expert_combine_join(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
                         weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float,
                         eps: float, residual: torch.Tensor, gain: torch.Tensor, alpha: float,
@@ -317,6 +367,7 @@ def dispatch_workspace_size(T: int, k: int, E: int) -> int:
     return int(load().moe_dispatch_workspace_size(T, k, E))
 
 
+@_traced
 def moe_dispatch(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0,
                  expert_offsets: Optional[torch.Tensor] = None, row_idx: Optional[torch.Tensor] = None,
                  row_token: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
@@ -354,6 +405,7 @@ def moe_dispatch(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0
     return expert_offsets, row_idx, row_token
 
 
+@_traced
 def moe_dispatch_noalloc(topk_ids: torch.Tensor, num_experts: int, expert_begin: int = 0,
                          expert_offsets: Optional[torch.Tensor] = None,
                          row_idx: Optional[torch.Tensor] = None,
@@ -385,6 +437,7 @@ def moe_dispatch_noalloc(topk_ids: torch.Tensor, num_experts: int, expert_begin:
     return expert_offsets, row_idx, row_token
 
 
+@_traced
 def router_weight_prepare(w: torch.Tensor, w3: Optional[torch.Tensor] = None, stream=None):
     """FP32 router weight [E, H] -> its three BF16 parts [3, E, H] (done once)."""
     _want(w, torch.float32, "w")
@@ -398,6 +451,7 @@ def router_weight_prepare(w: torch.Tensor, w3: Optional[torch.Tensor] = None, st
     return w3
 
 
+@_traced
 def router_logits(x: torch.Tensor, w3: torch.Tensor, scale: float = 1.0,
                   logits: Optional[torch.Tensor] = None, stream=None):
     """Router projection on the tensor cores: logits float32 [T, E] =
@@ -424,6 +478,7 @@ def finalize_ar_workspace_size(world: int, T_max: int, H: int) -> int:
     return int(load().finalize_ar_workspace_size(world, T_max, H))
 
 
+@_traced
 def finalize_ar_workspace_init(workspace, world: int, T_max: int, H: int, stream=None) -> None:
     """Zero a workspace's call counter and flags (a tensor or a device address)."""
     ptr = _ptr(workspace) if isinstance(workspace, torch.Tensor) else ctypes.c_void_p(int(workspace))
@@ -446,6 +501,7 @@ def _far_rank_check(fn, expert_out, row_idx, weights, norm_w, out):
         raise ValueError(f"{fn}: shape mismatch")
 
 
+@_traced
 def expert_finalize_allreduce(expert_out: torch.Tensor, num_rows: int, row_idx: torch.Tensor,
                               weights: torch.Tensor, norm_w: torch.Tensor, gain_center: float, eps: float,
                               workspaces, rank: int, T_max: int, out: Optional[torch.Tensor] = None,
@@ -472,6 +528,7 @@ def expert_finalize_allreduce(expert_out: torch.Tensor, num_rows: int, row_idx: 
     return out
 
 
+@_traced
 def expert_finalize_allreduce_local(expert_outs, num_rows, row_idx, weights, norm_w: torch.Tensor,
                                     gain_center: float, eps: float, workspaces, T_max: int, outs=None,
                                     stream=None):

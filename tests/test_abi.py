@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import expert_combine_b200 as eb
 
@@ -140,3 +141,18 @@ def test_finalize_ar_sizes_without_device_work():
     assert eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 8, 4)
     assert not eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 8, 9)
     assert not eb.supported(eb.STAGE_FINALIZE_AR, 128, 8192, 0, 33, 4)
+
+
+def test_trace_context_nests_and_keeps_names():
+    assert not eb.tracing()
+    with eb.trace():
+        assert eb.tracing()
+        with eb.trace():
+            assert eb.tracing()
+        assert eb.tracing()
+    assert not eb.tracing()
+    assert eb.expert_combine.__name__ == "expert_combine" and eb.expert_combine.__doc__
+    # inside a trace, a call that fails its argument checks still raises and closes its range
+    with eb.trace():
+        with pytest.raises((TypeError, ValueError)):
+            eb.moe_route(torch.zeros(4, 8), torch.zeros(8), torch.zeros(4, dtype=torch.int32), 2)
