@@ -3,6 +3,17 @@
  * layer on NVIDIA B200 (sm_100a): router gate, pre-expert RMSNorm fused with
  * NVFP4 quantisation, post-expert norm + weighted combine, gated residual join.
  *
+ * Entry points: moe_route, norm_quant_nvfp4, moe_route_norm_quant (both
+ * pre-expert stages in one call), expert_combine, residual_join,
+ * expert_combine_join (the combine with the join fused), moe_dispatch and
+ * moe_dispatch_noalloc (expert-grouped rows of the routing entries),
+ * router_weight_prepare and router_logits (the router projection),
+ * expert_finalize_allreduce and expert_finalize_allreduce_local (the combine
+ * of an expert-parallel layer fused with its tensor-parallel all-reduce) with
+ * their workspace calls and the mb_ipc_* peer-memory helpers; queries
+ * moe_boundary_supported, moe_route_norm_quant_kernels, the workspace sizes,
+ * mb_last_error and mb_device_status.
+ *
  * Library: libmoe_boundary.so (CUDA runtime only; no PyTorch types).
  *
  * Conventions shared by every entry point
@@ -11,7 +22,9 @@
  *    contiguous; every base pointer must be 16-byte aligned.  BF16 values are
  *    passed as uint16_t bit patterns, E4M3 and packed E2M1 as uint8_t.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
- *    only enqueued; nothing is synchronised, allocated or freed.
+ *    only enqueued; nothing is synchronised, allocated or freed (except by the
+ *    calls whose job that is: mb_ipc_alloc / mb_ipc_free / mb_ipc_open /
+ *    mb_ipc_close, and mb_device_status, which synchronises to read its word).
  *  - Return value: MB_OK, or an error code.  Arguments are checked before
  *    anything is enqueued, so on an error nothing runs; mb_last_error()
  *    returns a message for the calling thread's most recent failure.
