@@ -46,7 +46,9 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # MB_ORACLE_LIB names another compiled copy of oracle.c to load
+            # instead (the mutation tests point it at deliberately broken ones)
+            lib = ctypes.CDLL(os.environ.get("MB_ORACLE_LIB") or build())
             P = ctypes.c_void_p
             i32, i64, f32 = ctypes.c_int, ctypes.c_int64, ctypes.c_float
             sig = {
