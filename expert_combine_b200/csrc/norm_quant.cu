@@ -40,10 +40,10 @@ struct FusedRouteArgs {
     float* weights;
 };
 
-// Router warps added to a wide norm-quant CTA (after its 16 row warps), two
-// per SM sub-partition; at 768 threads the kernel fits in 80 registers a
+// Router warps added to a wide norm-quant CTA (after its 16 row warps), three
+// per SM sub-partition; at 896 threads the kernel fits in 72 registers a
 // thread without spilling.
-constexpr int kFusedRouterWarps = 8;
+constexpr int kFusedRouterWarps = 12;
 // The router warps use the small selection path with 8 scores per lane.
 constexpr int kFusedRouteMaxExperts = 256;
 
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // a shared-memory table read without bank conflicts.
 //
 // ROUTE: the CTA carries router warps after its row warps; they route the same
-// M tokens (two per warp iteration, statically interleaved over the grid's
+// M tokens (one per warp iteration, statically interleaved over the grid's
 // router warps) in the issue slots and registers the streaming row warps
 // leave free, so the latency-bound router adds little to the bandwidth-bound
 // norm-quant.  The router warps touch no shared memory and no barrier after
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     if constexpr (ROUTE) {
         constexpr int RW = kFusedRouterWarps;
         if (warp >= NTEAM * TW) {
-            route_pairs<8>(ra.logits, ra.bias, ra.mask, a.M, ra.E, ra.k, ra.ids, ra.weights,
+            route_singles<8>(ra.logits, ra.bias, ra.mask, a.M, ra.E, ra.k, ra.ids, ra.weights,
                            static_cast<int>(blockIdx.x) * RW + (warp - NTEAM * TW),
                            static_cast<int>(gridDim.x) * RW, lane);
             return;

@@ -388,4 +388,42 @@ __device__ __forceinline__ void route_pairs(const float* __restrict__ logits, co
     }
 }
 
+// One token per warp iteration (t, t + nwarps, ...), for the router warps of
+// the fused norm-quant kernel: with a fixed number of warps each warp routes
+// several tokens, and one selection chain at a time measured faster there
+// than two interleaved (or than the next token's logits held in registers).
+// The next token's mask byte is read at the end of each iteration.
+template <int MODE>
+__device__ __forceinline__ void route_singles(const float* __restrict__ logits, const float* __restrict__ bias,
+                                              const uint8_t* __restrict__ mask, int T, int E, int k,
+                                              int32_t* __restrict__ ids, float* __restrict__ weights, int warp,
+                                              int nwarps, int lane) {
+    const bool vec = (E & 3) == 0;
+    int t = warp;
+    if (t >= T) return;
+    bool valid = mask[t] != 0;
+    float lv[MODE];
+#pragma unroll
+    for (int i = 0; i < MODE; ++i) lv[i] = 0.0f;
+    for (;;) {
+        const int tn = t + nwarps;
+        if (valid) load_logits<MODE>(logits + static_cast<size_t>(t) * E, E, lane, vec, lv);
+        int32_t* id_row = ids + static_cast<size_t>(t) * k;
+        float* w_row = weights + static_cast<size_t>(t) * k;
+        if (!valid) {
+            if (lane < k) {
+                id_row[lane] = -1;
+                w_row[lane] = 0.0f;
+            }
+        } else {
+            uint32_t pick_key = 0u, pick_id = 0u;
+            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+            route_write(logits + static_cast<size_t>(t) * E, k, lane, pick_id, id_row, w_row);
+        }
+        if (tn >= T) break;
+        t = tn;
+        valid = mask[t] != 0;
+    }
+}
+
 }  // namespace mb
