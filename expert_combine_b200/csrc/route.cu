@@ -1,4 +1,4 @@
-// route.cu -- stage 1, the sigmoid router gate (one warp per token).
+// route.cu -- stage 1, the sigmoid router gate (one token per warp iteration).
 //
 // Computes, per valid token t (TensorRT-LLM PR 21356 "Muse Spark Open decoder
 // fast paths", description, Routing; lmdeploy PR 4835 "MoE gate v2", token
@@ -47,30 +47,11 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
     const bool vec = (E & 3) == 0;
 
-    // one token per warp when the batch fits the grid's warps (few tokens:
-    // the shortest chain per token), else two per warp iteration
+    // one token per warp iteration: each token's selection is one dependent
+    // chain of warp reductions, and more warps with one chain each measured
+    // faster than fewer warps interleaving two
     if constexpr (MODE > 0) {
-        if (BESIDE || T <= nwarps) {
-            for (int t = warp; t < T; t += nwarps) {
-                int32_t* id_row = ids + static_cast<size_t>(t) * k;
-                float* w_row = weights + static_cast<size_t>(t) * k;
-                if (mask[t] == 0) {
-                    if (lane < k) {
-                        id_row[lane] = -1;
-                        w_row[lane] = 0.0f;
-                    }
-                    continue;
-                }
-                const float* l = logits + static_cast<size_t>(t) * E;
-                float lv[MODE];
-                load_logits<MODE>(l, E, lane, vec, lv);
-                uint32_t pick_key = 0u, pick_id = 0u;
-                select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
-                route_write(l, k, lane, pick_id, id_row, w_row);
-            }
-        } else {
-            route_pairs<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
-        }
+        route_singles<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
     } else {
         for (int t = warp; t < T; t += nwarps) {
             int32_t* id_row = ids + static_cast<size_t>(t) * k;
@@ -100,10 +81,7 @@ cudaError_t launch_route_cfg(const float* logits, const float* bias, const uint8
     const int warps_per_cta = threads / 32;
     // scores per lane, rounded up to whole 128-bit loads
     const int epl = (per_lane + 3) / 4 * 4;
-    // the small path routes two tokens per warp iteration, or one per warp when
-    // a grid of one token per warp fits under the cap
-    int grid = (T + warps_per_cta - 1) / warps_per_cta;
-    if (epl <= 16 && !BESIDE && grid > grid_cap) grid = (T + 2 * warps_per_cta - 1) / (2 * warps_per_cta);
+    int grid = (T + warps_per_cta - 1) / warps_per_cta;   // one token per warp, up to the cap
     if (grid > grid_cap) grid = grid_cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

@@ -181,80 +181,6 @@ __device__ __forceinline__ void select_small(const float (&lv)[EPL], const float
     }
 }
 
-// Two tokens at once (independent selection chains interleaved round by
-// round); tokens that are absent or masked are given all-zero keys and their
-// picks are ignored by the caller.
-template <int EPL>
-__device__ __forceinline__ void select_small2(const float (&la)[EPL], const float (&lb)[EPL], bool va, bool vb,
-                                              const float* bias, int E, int k, int lane, bool vec,
-                                              uint32_t& pick_a, uint32_t& pick_b) {
-    uint32_t ka[EPL], kb[EPL];
-#pragma unroll
-    for (int u = 0; u < EPL / 4; ++u) {
-        const int q = lane + 32 * u;
-        float4 b;
-        if (vec && 4 * q + 3 < E) {
-            b = __ldg(reinterpret_cast<const float4*>(bias) + q);
-        } else {
-            b.x = 4 * q + 0 < E ? __ldg(bias + 4 * q + 0) : 0.0f;
-            b.y = 4 * q + 1 < E ? __ldg(bias + 4 * q + 1) : 0.0f;
-            b.z = 4 * q + 2 < E ? __ldg(bias + 4 * q + 2) : 0.0f;
-            b.w = 4 * q + 3 < E ? __ldg(bias + 4 * q + 3) : 0.0f;
-        }
-        const float bb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool in = 4 * q + i < E;
-            ka[4 * u + i] = (va && in) ? score_key(__fadd_rn(sigmoid_fixed(la[4 * u + i]), bb[i])) : 0u;
-            kb[4 * u + i] = (vb && in) ? score_key(__fadd_rn(sigmoid_fixed(lb[4 * u + i]), bb[i])) : 0u;
-        }
-    }
-    LaneTop2<EPL> ca, cb;
-    ca.init(ka, lane);
-    cb.init(kb, lane);
-    for (int j = 0; j < k; ++j) {
-        const uint32_t ma = warp_max_u32(ca.k1);
-        const uint32_t mb = warp_max_u32(cb.k1);
-        const uint32_t wa = warp_min_u32(ca.k1 == ma ? ca.id1 : 0xffffffffu);
-        const uint32_t wb = warp_min_u32(cb.k1 == mb ? cb.id1 : 0xffffffffu);
-        if (ca.k1 == ma && ca.id1 == wa) ca.pop(ka, lane);
-        if (cb.k1 == mb && cb.id1 == wb) cb.pop(kb, lane);
-        if (lane == j) {
-            pick_a = wa;
-            pick_b = wb;
-        }
-    }
-}
-
-// Picks of two tokens written together (lane j < k holds pick j of each);
-// a token that is absent (t >= T) is skipped, a masked one gets -1 / 0.
-__device__ __forceinline__ void route_write2(const float* logits, int E, int k, int lane, int ta, int tb,
-                                             bool pa, bool pb, bool va, bool vb, uint32_t id_a, uint32_t id_b,
-                                             int32_t* ids, float* weights) {
-    const float* la = logits + static_cast<size_t>(ta) * E;
-    const float* lb = logits + static_cast<size_t>(tb) * E;
-    float sa = 0.0f, sb = 0.0f;
-    if (lane < k) {
-        if (va) sa = sigmoid_fixed(__ldg(la + id_a));
-        if (vb) sb = sigmoid_fixed(__ldg(lb + id_b));
-    }
-    float Sa = 0.0f, Sb = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        Sa = __fadd_rn(Sa, __shfl_sync(0xffffffffu, sa, j));
-        Sb = __fadd_rn(Sb, __shfl_sync(0xffffffffu, sb, j));
-    }
-    if (lane < k) {
-        if (pa) {
-            ids[static_cast<size_t>(ta) * k + lane] = va ? static_cast<int32_t>(id_a) : -1;
-            weights[static_cast<size_t>(ta) * k + lane] = va ? __fdiv_rn(sa, Sa) : 0.0f;
-        }
-        if (pb) {
-            ids[static_cast<size_t>(tb) * k + lane] = vb ? static_cast<int32_t>(id_b) : -1;
-            weights[static_cast<size_t>(tb) * k + lane] = vb ? __fdiv_rn(sb, Sb) : 0.0f;
-        }
-    }
-}
-
 // The picks' unbiased sigmoids, renormalised in pick order (lane j < k holds
 // pick j), written with the ids.
 __device__ __forceinline__ void route_write(const float* l, int k, int lane, uint32_t pick_id, int32_t* id_row,
@@ -340,59 +266,11 @@ __device__ __forceinline__ void route_token_list(const float* l, const float* bi
 }
 
 
-// Two tokens per warp iteration (t and t + nwarps), for the small path
-// (E <= 32 * MODE).  The next pair's mask bytes and logits are loaded one
-// iteration ahead, so a warp that routes many tokens keeps a load in flight
-// while it selects.
-template <int MODE>
-__device__ __forceinline__ void route_pairs(const float* __restrict__ logits, const float* __restrict__ bias,
-                                            const uint8_t* __restrict__ mask, int T, int E, int k,
-                                            int32_t* __restrict__ ids, float* __restrict__ weights, int warp,
-                                            int nwarps, int lane) {
-    const bool vec = (E & 3) == 0;
-    int t = warp;
-    if (t >= T) return;
-    bool va = mask[t] != 0;
-    bool pb = t + nwarps < T;
-    bool vb = pb && mask[t + nwarps] != 0;
-    float la[MODE], lb[MODE];
-#pragma unroll
-    for (int i = 0; i < MODE; ++i) la[i] = lb[i] = 0.0f;
-    if (va) load_logits<MODE>(logits + static_cast<size_t>(t) * E, E, lane, vec, la);
-    if (vb) load_logits<MODE>(logits + static_cast<size_t>(t + nwarps) * E, E, lane, vec, lb);
-    for (;;) {
-        const int tn = t + 2 * nwarps;
-        const bool pn = tn < T;
-        const bool pnb = tn + nwarps < T;
-        const bool vna = pn && mask[tn] != 0;
-        const bool vnb = pnb && mask[tn + nwarps] != 0;
-        float na[MODE], nb[MODE];
-#pragma unroll
-        for (int i = 0; i < MODE; ++i) na[i] = nb[i] = 0.0f;
-        if (vna) load_logits<MODE>(logits + static_cast<size_t>(tn) * E, E, lane, vec, na);
-        if (vnb) load_logits<MODE>(logits + static_cast<size_t>(tn + nwarps) * E, E, lane, vec, nb);
-        uint32_t ida = 0u, idb = 0u;
-        select_small2<MODE>(la, lb, va, vb, bias, E, k, lane, vec, ida, idb);
-        const int tb = pb ? t + nwarps : t;
-        route_write2(logits, E, k, lane, t, tb, true, pb, va, vb, ida, idb, ids, weights);
-        if (!pn) break;
-        t = tn;
-        va = vna;
-        vb = vnb;
-        pb = pnb;
-#pragma unroll
-        for (int i = 0; i < MODE; ++i) {
-            la[i] = na[i];
-            lb[i] = nb[i];
-        }
-    }
-}
-
-// One token per warp iteration (t, t + nwarps, ...), for the router warps of
-// the fused norm-quant kernel: with a fixed number of warps each warp routes
-// several tokens, and one selection chain at a time measured faster there
-// than two interleaved (or than the next token's logits held in registers).
-// The next token's mask byte is read at the end of each iteration.
+// One token per warp iteration (t, t + nwarps, ...) on the small path
+// (E <= 32 * MODE), for the router kernels and the router warps of the fused
+// norm-quant kernel: one selection chain at a time measured faster than two
+// interleaved (or than the next token's logits held in registers).  The next
+// token's mask byte is read at the end of each iteration.
 template <int MODE>
 __device__ __forceinline__ void route_singles(const float* __restrict__ logits, const float* __restrict__ bias,
                                               const uint8_t* __restrict__ mask, int T, int E, int k,
