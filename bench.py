@@ -87,7 +87,8 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,clocks.mem,"
+              "power.limit")
 
     def __init__(self, device_index):
         self.idx = device_index
@@ -124,9 +125,14 @@ class ClockSampler:
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        num = lambda v: v.replace(".", "").isdigit()
+        mem = [float(r[9]) for r in rows if len(r) > 9 and num(r[9])]
+        pw = [float(r[3]) for r in rows if num(r[3])]
+        lim = [float(r[10]) for r in rows if len(r) > 10 and num(r[10])]
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "mem_mhz": statistics.median(mem) if mem else None,
+                "power_w_max": max(pw) if pw else None, "power_limit_w": min(lim) if lim else None}
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -362,6 +368,8 @@ def run_ours(args, info):
             "gpu_launches": (pre_kernels + 1) * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
+                       "mem_mhz": clk.get("mem_mhz"), "power_w_max": clk.get("power_w_max"),
+                       "power_limit_w": clk.get("power_limit_w"),
                        "timed_wall_s": t_wall},
         }
         print(json.dumps(result), flush=True)
