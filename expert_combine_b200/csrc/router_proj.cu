@@ -12,17 +12,21 @@
 // weight is prepared once into three BF16 parts, w = w1 + w2 + w3 + d with
 // w1 = bf16(w), w2 = bf16(w - w1), w3 = bf16(w - w1 - w2) (each remainder is
 // exact in FP32) and |d| <= 2^-27 |w|.  A product of two BF16 values is exact
-// in FP32, so x W^T = x w1^T + x w2^T + x w3^T, three MMAs per K step,
-// accumulated in FP32 by the tensor core.
+// in FP32, so x W^T = x w1^T + x w2^T + x w3^T.  The three parts of a CTA's 16
+// experts sit side by side as one 48-row B operand, so each K step is a single
+// MMA (M = 128, N = 48) that reads the x slice from shared memory once; the
+// tensor core accumulates each part in its own 16 FP32 columns, and the
+// epilogue adds them, the two small parts first: w1 + (w2 + w3).
 //
 // Work split (one M tile of 128 token rows per grid row; rows >= T read as
 // zero): each CTA owns 16 experts and one of C contiguous K chunks, C <= 8
 // CTAs of a thread-block cluster.  One thread streams the chunk's slabs of
 // 64 K elements with TMA into a 4-stage ring (x: 128 rows x 128 bytes, the
 // three weight parts: 16 rows x 128 bytes each, all 128-byte swizzled, which
-// is the K-major layout the MMA reads); another thread issues each slab's 12
-// MMAs (4 K steps of 16 x 3 parts, M = 128, N = 16) into a 128 x 16 FP32
-// accumulator in tensor memory and hands the stage back with tcgen05.commit.
+// is the K-major layout the MMA reads, the parts back to back); another thread
+// issues each slab's 4 MMAs (K steps of 16, M = 128, N = 48) into a 128 x 48
+// FP32 accumulator in tensor memory and hands the stage back with
+// tcgen05.commit.
 // No CTA-wide barrier runs inside the K loop.  The C partial accumulators are
 // then summed across the cluster in rank order through distributed shared
 // memory (no atomics: the same result run to run), scaled, and written for the
@@ -42,9 +46,12 @@ constexpr int kRpSlabK = 64;              // K elements per slab (one 128-byte s
 constexpr int kRpStages = 4;
 constexpr int kRpXTile = kRpM * 128;      // 16 KB
 constexpr int kRpWTile = kRpN * 128;      // 2 KB per weight part
-constexpr int kRpStageBytes = kRpXTile + 3 * kRpWTile;
+constexpr int kRpStageBytes = kRpXTile + 3 * kRpWTile;   // parts back to back: one 48-row B operand
 constexpr size_t kRpSmemBytes = 1024 + kRpStages * kRpStageBytes + kRpM * kRpN * 4;
-constexpr int kRpTmemCols = 32;           // allocation unit >= N
+constexpr int kRpNParts = 3 * kRpN;       // MMA N: the three weight parts side by side
+constexpr int kRpTmemCols = 64;           // allocation unit >= kRpNParts
+static_assert(kRpNParts % 16 == 0 && kRpNParts <= 256, "an M = 128 MMA takes N in steps of 16 up to 256");
+static_assert(kRpNParts <= kRpTmemCols, "the accumulator fits its tensor-memory allocation");
 
 struct RouterProjArgs {
     float* logits;        // [T, E] FP32
@@ -111,8 +118,8 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 }
 
 // Instruction descriptor: FP32 accumulator, BF16 A and B, both K-major,
-// N = kRpN, M = kRpM.
-constexpr uint32_t kRpIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kRpN >> 3) << 17) |
+// N = kRpNParts, M = kRpM.
+constexpr uint32_t kRpIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kRpNParts >> 3) << 17) |
                               (static_cast<uint32_t>(kRpM >> 4) << 24);
 
 template <int C>
@@ -187,13 +194,9 @@ __global__ void __launch_bounds__(kRpThreads) router_proj_kernel(const __grid_co
             tc_fence_after();
             const uint32_t sa = smem_addr(stages + s * kRpStageBytes);
 #pragma unroll
-            for (int ks = 0; ks < kRpSlabK / 16; ++ks) {   // K steps of 16 BF16 = 32 bytes
-                const uint64_t ad = smem_desc_sw128(sa + 32u * ks);
-#pragma unroll
-                for (int p = 0; p < 3; ++p)
-                    mma_bf16(tmem_d, ad, smem_desc_sw128(sa + kRpXTile + p * kRpWTile + 32u * ks), kRpIdesc,
-                             (j | ks | p) != 0 ? 1u : 0u);
-            }
+            for (int ks = 0; ks < kRpSlabK / 16; ++ks)   // K steps of 16 BF16 = 32 bytes; B = parts 0..2
+                mma_bf16(tmem_d, smem_desc_sw128(sa + 32u * ks), smem_desc_sw128(sa + kRpXTile + 32u * ks), kRpIdesc,
+                         (j | ks) != 0 ? 1u : 0u);
             mma_commit(&empty[s]);
         }
         s_consumed = j;
@@ -209,11 +212,17 @@ __global__ void __launch_bounds__(kRpThreads) router_proj_kernel(const __grid_co
             mbar_wait_bounded(&full[j % kRpStages], static_cast<uint32_t>((j / kRpStages) & 1), 8u);
     tc_fence_after();
 
-    // partial accumulator: warp w holds token rows 32w .. 32w + 31
-    float v[16];
-    tmem_ld16(tmem_d + (static_cast<uint32_t>(32 * warp) << 16), v);
+    // partial accumulator: warp w holds token rows 32w .. 32w + 31; part p of
+    // expert n in column 16 p + n
+    const uint32_t trow = tmem_d + (static_cast<uint32_t>(32 * warp) << 16);
+    float v[16], u[16];
+    tmem_ld16(trow + 16u, v);
+    tmem_ld16(trow + 32u, u);
 #pragma unroll
-    for (int n = 0; n < kRpN; ++n) part[(32 * warp + lane) * kRpN + n] = complete ? v[n] : 0.0f;
+    for (int n = 0; n < kRpN; ++n) u[n] = v[n] + u[n];
+    tmem_ld16(trow, v);
+#pragma unroll
+    for (int n = 0; n < kRpN; ++n) part[(32 * warp + lane) * kRpN + n] = complete ? v[n] + u[n] : 0.0f;
     tc_fence_before();
     if constexpr (C > 1) {
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
