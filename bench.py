@@ -195,13 +195,25 @@ def time_oracle(case_host, tokens, budget_s=15.0):
     return len(tokens) / med, cores, reps, med
 
 
+def prefill_config(case, world):
+    """The `config` of the JSON line: the prefill workload, the same on both arms."""
+    from expert_combine_b200 import synth
+    idx_h = synth.host(case.row_idx)
+    return {"workload": f"prefill T={case.T} H={case.H} E={case.E} k={case.k} (route+norm-quant+combine)",
+            "tokens_per_rank": case.T, "hidden": case.H, "experts": case.E, "top_k": case.k,
+            "expert_rows": case.R, "valid_tokens": int(synth.host(case.mask).sum()),
+            "valid_slots": int(((idx_h >= 0) & (idx_h < case.R)).sum()), "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2 (1.2 GB per step), no flush"}
+
+
 # ---------------------------------------------------------------------------- reference arm
 def run_reference(args, info):
     if info.rank != 0:
         return 0
     from expert_combine_b200 import synth
-    case = synth.make_case(WORKLOAD, device="cuda" if torch.cuda.is_available() else "cpu")
-    n_sample = 256
+    case = synth.make_case(WORKLOAD, device="cuda" if torch.cuda.is_available() else "cpu",
+                           seed=shard.rank_seed(synth.SEEDS[WORKLOAD], info), T=args.tokens)
+    n_sample = min(256, case.T)
     tokens, ch = host_sample(case, n_sample, seed=1)
     import oracle
     cores = oracle.get_threads()
@@ -219,10 +231,10 @@ def run_reference(args, info):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "prefill T=8192 H=8192 E=256 k=8 (oracle on a token sample)",
-                   "sample_tokens": n_sample},
+        "config": prefill_config(case, info.world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n_sample} of 8192 tokens per step, all three stages"},
+                         "sample": f"{n_sample} of {case.T} tokens per step (all three stages), "
+                                   f"scaled to the metric's unit"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -311,7 +323,6 @@ def run_ours(args, info):
     b_route, b_nq, b_cmb = bytes_per_token(H, E, k)
     idx_h = synth.host(case.row_idx)
     valid_slots = int(((idx_h >= 0) & (idx_h < case.R)).sum())
-    valid_tokens = int(synth.host(case.mask).sum())
     cmb_bytes_nominal = T * b_cmb
     cmb_bytes_net = valid_slots * 2 * H + T * (8 * k + 2 * H)
     step_bytes_nominal = T * (b_route + b_nq + b_cmb)
@@ -343,11 +354,7 @@ def run_ours(args, info):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"prefill T={T} H=8192 E=256 k=8 (route+norm-quant+combine)",
-                       "tokens_per_rank": T, "hidden": H, "experts": E, "top_k": k,
-                       "expert_rows": case.R, "valid_tokens": valid_tokens,
-                       "valid_slots": valid_slots, "parallelism": f"dp{world}",
-                       "l2": "inputs larger than L2 (1.2 GB per step), no flush"},
+            "config": prefill_config(case, world),
             "hbm": {"step_bytes_nominal": step_bytes_nominal,
                     "step_gbs": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9,
                     "frac_of_8tbs": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
