@@ -179,6 +179,23 @@ def host_sample(case, n_tokens, seed=0):
                         post_gc=case.post_gc)
 
 
+def near_threshold_report(case, packed, sf):
+    """NVFP4 values of the whole batch whose FP32 pre-quantisation value (or
+    the scale's FP32 argument) lies within one ulp of a rounding threshold,
+    counted by the oracle over every token, and how many of the GPU's codes and
+    scales differ from the oracle's (part of the CPU-baseline leg: the only
+    place the benchmark runs the oracle)."""
+    import oracle
+    from expert_combine_b200 import synth
+    p_o, s_o, near_ = oracle.norm_quant(synth.host(case.x), case.T, case.H, case.tp, synth.host(case.norm_w),
+                                        case.gc, case.eps, float(synth.host(case.gs)[0]), return_near=True)
+    return {"codes_near": near_[0], "scales_near": near_[1], "codes": case.T * case.H,
+            "scales": case.T * case.H // 16,
+            "packed_bytes_differing": int((synth.host(packed) != p_o).sum()),
+            "scales_differing": int((synth.host(sf) != s_o).sum()),
+            "how": "oracle over all tokens of the step's batch; the GPU's outputs of the last timed step"}
+
+
 def time_oracle(case_host, tokens, budget_s=15.0):
     import oracle
     cores = oracle.get_threads()
@@ -332,6 +349,11 @@ def run_ours(args, info):
     disp = None if args.no_dispatch else run_dispatch(eb, ids, E, dev, reps=max(5, min(args.steps, 200)))
     dec = None if args.no_decode else run_decode(eb, dev, reps=max(5, min(args.steps, 100)))
     far = None if args.no_finalize_ar else run_finalize_ar(eb, dev, peak, reps=max(5, min(args.steps, 100)))
+    legs = {}
+    if not args.no_legs:
+        for name in ("large_e", "wide_topk"):
+            legs[name] = run_leg(eb, name, dev, steps=max(5, min(args.steps, 50)), warmup=args.warmup, peak=peak)
+            torch.cuda.empty_cache()
 
     # end to end through the same calls with host buffers (pinned), copies inside
     e2e = None if args.no_e2e else run_e2e(eb, case, dev, stream, ids, w, packed, sf, out,
@@ -341,6 +363,7 @@ def run_ours(args, info):
     result = None
     if rank == 0:
         cpu = None
+        near = None
         if world == 1 and not args.no_cpu_baseline and T >= 512:
             n_sample = 512
             tokens, ch = host_sample(case, n_sample, seed=2)
@@ -348,6 +371,7 @@ def run_ours(args, info):
             cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                    "sample": f"{n_sample} of 8192 tokens (all three stages), median of {reps} "
                              f"runs of {med:.2f} s"}
+            near = near_threshold_report(case, packed, sf)
         clk = clocks.summary()
         result = {
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -372,6 +396,9 @@ def run_ours(args, info):
             "dispatch": disp,
             "decode": dec,
             "finalize_allreduce": far,
+            "large_e": legs.get("large_e"),
+            "wide_topk": legs.get("wide_topk"),
+            "near_threshold": near,
             "gpu_launches": (pre_kernels + 1) * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
                        "reasons": clk["reasons"], "samples": clk["samples"],
@@ -515,6 +542,98 @@ def run_finalize_ar(eb, dev, peak, reps):
             "how": f"{reps} calls per CUDA graph, one replay between two events"}
 
 
+def run_leg(eb, name, dev, steps, warmup, peak):
+    """Another workload of the pages at its full size, as one step per
+    iteration: moe_route_norm_quant, then (wide top-k) the dispatch of the
+    router's ids, then expert_combine with the router's weights.  The step's
+    time (K back-to-back steps between two events) and each stage alone (K
+    back-to-back launches), against the algorithmic bytes of each stage."""
+    from expert_combine_b200 import synth
+    case = synth.make_case(name, device=dev, seed=synth.SEEDS[name])
+    T, H, E, k = case.T, case.H, case.E, case.k
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    packed = torch.empty(T, H // 2, dtype=torch.uint8, device=dev)
+    sf = torch.empty(T, H // 16, dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    chained = name == "wide_topk"          # stages end to end: the combine reads the dispatched rows
+    if chained:
+        offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        row_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        row_tok = torch.empty(T * k, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(16, eb.dispatch_workspace_size(T, k, E)), dtype=torch.uint8, device=dev)
+    else:
+        row_idx = case.row_idx
+    stream = torch.cuda.current_stream(dev)
+
+    def route():
+        eb.moe_route(case.logits, case.bias, case.mask, k, ids, w)
+
+    def norm_quant():
+        eb.norm_quant_nvfp4(case.x, T, case.norm_w, case.gc, case.eps, case.gs, tp=case.tp, packed=packed, sf=sf)
+
+    def pre():
+        eb.moe_route_norm_quant(case.logits, case.bias, case.mask, k, case.x, case.norm_w, case.gc, case.eps,
+                                case.gs, tp=case.tp, topk_ids=ids, topk_weights=w, packed=packed, sf=sf)
+
+    def dispatch():
+        eb.moe_dispatch(ids, E, 0, offs, row_idx, row_tok, ws)
+
+    def combine():
+        eb.expert_combine(case.expert_out, case.R, row_idx, w, case.post_w, case.post_gc, case.eps, out=out)
+
+    def step():
+        pre()
+        if chained:
+            dispatch()
+        combine()
+
+    def per_call_ms(fn, n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n):
+            fn()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    step_ms = per_call_ms(step, steps)
+    stages = {"route": route, "norm_quant": norm_quant, "route_norm_quant": pre}
+    if chained:
+        stages["dispatch"] = dispatch
+    stages["combine"] = combine
+    stage_us = {key: per_call_ms(fn, steps) * 1e3 for key, fn in stages.items()}
+    if eb.device_status() != 0:
+        raise RuntimeError(f"{name}: a kernel reported a wait timeout")
+
+    b_route, b_nq, b_cmb = bytes_per_token(H, E, k)
+    idx_h = synth.host(row_idx)
+    valid_slots = int(((idx_h >= 0) & (idx_h < case.R)).sum())
+    bytes_ = {"route": T * b_route, "norm_quant": T * b_nq, "route_norm_quant": T * (b_route + b_nq),
+              "dispatch": 12 * T * k,
+              "combine": valid_slots * 2 * H + T * (8 * k + 2 * H)}
+    stage_rep = {}
+    for key, us in stage_us.items():
+        gbs = bytes_[key] / (us * 1e-6) / 1e9
+        stage_rep[key] = {"us": us, "bytes": bytes_[key], "gbs": gbs, "frac_of_measured_hbm": gbs / peak}
+    step_bytes = T * (b_route + b_nq + b_cmb)
+    step_gbs = step_bytes / (step_ms * 1e-3) / 1e9
+    layout = f"rank-block [{case.tp}, {T}, {H // case.tp}]" if case.tp > 1 else "contiguous"
+    return {"workload": f"{name} T={T} H={H} E={E} k={k}, norm-quant input {layout}"
+                        + (", route -> dispatch -> combine end to end" if chained else ""),
+            "tokens_per_s": T / (step_ms * 1e-3), "ms_per_step": step_ms,
+            "step_bytes_nominal": step_bytes, "bytes_per_token": b_route + b_nq + b_cmb,
+            "step_gbs": step_gbs, "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS, "frac_of_measured": step_gbs / peak,
+            "stages": stage_rep, "valid_slots": valid_slots,
+            "how": f"{steps} back-to-back steps between two events; each stage alone the same way",
+            "gpu_launches_per_step": (eb.route_norm_quant_kernels(T, H, E, k, tp=case.tp)
+                                      + (1 if not chained else 1 + (1 if T * k <= 4096 else
+                                                                    (2 if T * k <= 32 * 4096 else 3))))}
+
+
 def run_e2e(eb, case, dev, stream, ids, w, packed, sf, out, pre_expert, steps):
     """Host inputs (pinned) -> device -> the boundary's calls -> host outputs,
     every step, through the public API.  Steps are pipelined over three
@@ -600,6 +719,8 @@ def main():
     ap.add_argument("--no-dispatch", action="store_true",
                     help="skip the separate timing of the dispatch step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the large-E gate and wide top-k workloads")
     ap.add_argument("--no-finalize-ar", action="store_true",
                     help="skip the separate timing of the finalize + all-reduce (one-device exchange)")
     ap.add_argument("--separate", action="store_true",

@@ -277,9 +277,14 @@ size_t moe_dispatch_workspace_size(int T, int k, int E) {
     return dispatch_workspace_bytes(static_cast<int64_t>(T) * k, E);
 }
 
-int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
-                 int32_t* row_idx, int32_t* row_token, void* workspace, size_t workspace_bytes, void* stream) {
-    const char* fn = "moe_dispatch";
+}  // extern "C"
+
+namespace mb {
+
+// The checks of moe_dispatch's arguments other than the workspace (shared with
+// moe_dispatch_noalloc, which must refuse the same inputs the same way).
+int check_dispatch(const char* fn, const int32_t* topk_ids, int T, int k, int expert_begin, int E,
+                   const int32_t* expert_offsets, const int32_t* row_idx, const int32_t* row_token) {
     if (T < 0 || k < 0 || E < 0 || expert_begin < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative argument", fn);
     if (static_cast<int64_t>(expert_begin) + E > INT32_MAX)
         return fail(MB_ERR_INVALID_ARG, "%s: expert_begin + E overflows int32", fn);
@@ -290,6 +295,18 @@ int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
         return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
     if (!aligned16(expert_offsets) || !aligned16(topk_ids) || !aligned16(row_idx) || !aligned16(row_token))
         return fail(MB_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", fn);
+    return MB_OK;
+}
+
+}  // namespace mb
+
+extern "C" {
+
+int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
+                 int32_t* row_idx, int32_t* row_token, void* workspace, size_t workspace_bytes, void* stream) {
+    const char* fn = "moe_dispatch";
+    const int st = check_dispatch(fn, topk_ids, T, k, expert_begin, E, expert_offsets, row_idx, row_token);
+    if (st != MB_OK) return st;
     const size_t need = dispatch_workspace_bytes(static_cast<int64_t>(T) * k, E);
     if (need > 0) {
         if (!workspace || workspace_bytes < need)

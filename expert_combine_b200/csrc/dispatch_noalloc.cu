@@ -14,7 +14,12 @@
 // The array lives in device memory for as long as the library is loaded, on
 // every GPU that loads it.  Its address is looked up once per device
 // (cudaGetSymbolAddress, with that device current) on the first call made on
-// that device; in host code the array's name only stands for it.
+// that device that succeeds; in host code the array's name only stands for it.
+// A failed lookup (for example an error left over from an earlier launch) is
+// not remembered: the next call looks again.  The remembered address belongs
+// to the device's context as it was at the lookup, so it assumes that context
+// lives as long as the process: after cudaDeviceReset the array is a new
+// allocation and this entry point must not be called again in that process.
 #include <mutex>
 
 #include "moe_boundary.h"
@@ -29,13 +34,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
 
 static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
-struct ScratchAddress {
-    std::once_flag once;
-    void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
 constexpr int kScratchDevices = 64;
-ScratchAddress g_scratch_address[kScratchDevices];
+std::mutex g_scratch_mutex;
+void* g_scratch_address[kScratchDevices] = {};   // null until a lookup on that device succeeded
 
 // Device address of g_dispatch_scratch on the current device.
 cudaError_t scratch_address(void** out) {
@@ -43,10 +44,15 @@ cudaError_t scratch_address(void** out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kScratchDevices) return cudaErrorInvalidDevice;
-    ScratchAddress& s = g_scratch_address[dev];
-    std::call_once(s.once, [&s] { s.err = cudaGetSymbolAddress(&s.ptr, g_dispatch_scratch); });
-    *out = s.ptr;
-    return s.err;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_address[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_address[dev] = p;
+    }
+    *out = g_scratch_address[dev];
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -56,16 +62,19 @@ cudaError_t scratch_address(void** out) {
 extern "C" int moe_dispatch_noalloc(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
                                     int32_t* expert_offsets, int32_t* row_idx, int32_t* row_token, void* stream) {
     using namespace mb;
+    const char* fn = "moe_dispatch_noalloc";
+    const int st = check_dispatch(fn, topk_ids, T, k, expert_begin, E, expert_offsets, row_idx, row_token);
+    if (st != MB_OK) return st;
     const size_t need = moe_dispatch_workspace_size(T, k, E);
     if (need > kNoAllocScratchBytes)
         return fail(MB_ERR_UNSUPPORTED,
-                    "moe_dispatch_noalloc: T=%d, k=%d, E=%d needs %zu bytes of scratch; the library's "
+                    "%s: T=%d, k=%d, E=%d needs %zu bytes of scratch; the library's "
                     "fixed array holds %zu (call moe_dispatch with a workspace instead)",
-                    T, k, E, need, kNoAllocScratchBytes);
+                    fn, T, k, E, need, kNoAllocScratchBytes);
     void* scratch = nullptr;
     if (need > 0) {
         const cudaError_t e = scratch_address(&scratch);
-        if (e != cudaSuccess) return cuda_status(e, "moe_dispatch_noalloc (scratch address)");
+        if (e != cudaSuccess) return cuda_status(e, "moe_dispatch_noalloc: scratch address");
     }
     return moe_dispatch(topk_ids, T, k, expert_begin, E, expert_offsets, row_idx, row_token, scratch,
                         need > 0 ? kNoAllocScratchBytes : 0, stream);

@@ -295,7 +295,9 @@ int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
  * nothing: its scratch is a fixed 1 MiB array compiled into the library,
  * which every GPU that loads the library holds until the process exits.
  *
- * Arguments, outputs and results are those of moe_dispatch (bit for bit).
+ * Arguments, outputs and results are those of moe_dispatch (bit for bit), and
+ * so are the argument checks and their status codes; only then is the size
+ * limit below checked.
  * Limit: the inputs must fit the array, (ceil(T * k / 4096) + 1) * E * 4 <=
  * 1 MiB (for example T * k up to about 4.19 M entries at E = 256, 413 K at
  * E = 2560); larger calls return MB_ERR_UNSUPPORTED without launching.
@@ -304,8 +306,11 @@ int moe_dispatch(const int32_t* topk_ids, int T, int k, int expert_begin, int E,
  * it and can return wrong rows.  Nothing in the array needs to start at zero
  * (each call writes every count it reads), and it keeps the last call's
  * counts.  The first call on a device looks up the array's device address
- * (synchronous, once per device, with that device current); make that first
- * call before any stream capture begins.
+ * (synchronous, with that device current) and keeps it once the lookup has
+ * succeeded (a failed lookup is retried by the next call); make that first
+ * call before any stream capture begins.  The kept address assumes the
+ * device's context lives as long as the process: after cudaDeviceReset, do
+ * not call this entry point again in the same process.
  */
 int moe_dispatch_noalloc(const int32_t* topk_ids, int T, int k, int expert_begin, int E, int32_t* expert_offsets,
                          int32_t* row_idx, int32_t* row_token, void* stream);

@@ -67,7 +67,7 @@ def _load():
                 "oc_norm_bf16": (None, [P, i32, i32, i32, P, f32, f32, P]),
                 "oc_norm_quant": (None, [P, i32, i32, i32, P, f32, f32, f32, P, P, P]),
                 "oc_combine": (None, [P, i64, i32, P, P, i32, i32, P, f32, f32, P]),
-                "oc_join": (None, [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32]),
+                "oc_join": (None, [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32, P]),
                 "oc_dispatch": (None, [P, i32, i32, i32, i32, P, P, P]),
                 "oc_router_logits": (None, [P, i32, i32, P, i32, f32, P, P]),
                 "oc_finalize_allreduce": (None, [P, P, i32, i32, P, P, i32, i32, P, f32, f32, P, P]),
@@ -269,10 +269,12 @@ def finalize_allreduce(expert_outs, Rs, row_idx, wt, w, gc: float, eps: float):
 
 
 def join(residual, branch, gain, alpha: float, beta: float, eps: float,
-         next_w=None, next_gc: float = 1.0, next_eps: float = 1e-6):
+         next_w=None, next_gc: float = 1.0, next_eps: float = 1e-6, return_normed: bool = False):
     """Gated residual join (+ next prenorm), Muse Spark Open fast paths.
 
-    Returns (new residual float32 [T, H], next prenorm uint16 [T, H] or None).
+    Returns (new residual float32 [T, H], next prenorm uint16 [T, H] or None),
+    and with ``return_normed`` also the BF16 bits of the normed branch term n
+    (uint16 [T, H]) that enters the residual as beta * n.
     """
     r = np.array(residual, dtype=np.float32, copy=True, order="C")
     T, H = r.shape
@@ -284,8 +286,11 @@ def join(residual, branch, gain, alpha: float, beta: float, eps: float,
     if next_w is not None:
         nw = _c(next_w, np.uint16)
         p = np.empty((T, H), np.uint16)
+    n = np.empty((T, H), np.uint16) if return_normed else None
     _load().oc_join(_ptr(r), _ptr(branch), _ptr(gain), float(alpha), float(beta), float(eps),
-                    _ptr(nw), float(next_gc), float(next_eps), _ptr(p), T, H)
+                    _ptr(nw), float(next_gc), float(next_eps), _ptr(p), T, H, _ptr(n))
+    if return_normed:
+        return r, p, n
     return r, p
 
 

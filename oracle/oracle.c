@@ -457,10 +457,12 @@ void oc_finalize_allreduce(const uint16_t* const* expert_out, const int64_t* R, 
  *   n  = bf16(g * inv_rms(g))                 (weightless RMSNorm)
  *   r' = alpha * r + beta * n                 (two products, one sum)
  * and, when next_w is not NULL,
- *   p  = bf16((r' * (next_gc + next_w)) * inv_rms(r'))  -> next_prenorm [T, H]. */
+ *   p  = bf16((r' * (next_gc + next_w)) * inv_rms(r'))  -> next_prenorm [T, H].
+ * normed (may be NULL) receives the BF16 bits of n [T, H]: the term whose
+ * BF16 step bounds the residual's tolerance. */
 void oc_join(float* residual, const uint16_t* branch, const uint16_t* gain, float alpha,
              float beta, float eps, const uint16_t* next_w, float next_gc, float next_eps,
-             uint16_t* next_prenorm, int T, int H) {
+             uint16_t* next_prenorm, int T, int H, uint16_t* normed) {
 #pragma omp parallel for schedule(dynamic, 4)
     for (int t = 0; t < T; ++t) {
         float* g = (float*)malloc(sizeof(float) * (size_t)H);
@@ -470,7 +472,9 @@ void oc_join(float* residual, const uint16_t* branch, const uint16_t* gain, floa
                                              oc_bf16_to_f32(branch[(size_t)t * H + h])));
         float inv = oc_inv_rms(oc_sumsq(g, H), H, eps);
         for (int h = 0; h < H; ++h) {
-            float n = oc_bf16_to_f32(oc_bf16_rn(g[h] * inv));
+            uint16_t nb = oc_bf16_rn(g[h] * inv);
+            float n = oc_bf16_to_f32(nb);
+            if (normed) normed[(size_t)t * H + h] = nb;
             float a = alpha * r[h];
             float b = beta * n;
             r[h] = a + b;

@@ -98,6 +98,17 @@ def test_bad_arguments_are_rejected_before_any_launch():
     assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, a, ctypes.c_size_t(need - 1), N) == 1
     assert lib.moe_dispatch(a, 8192, 8, 0, 256, a, a, a, odd, ctypes.c_size_t(need), N) == 1
     assert "aligned" in eb.last_error()
+    # the no-allocation dispatch refuses bad arguments exactly as moe_dispatch
+    # does, before its own size limit, and refuses too large inputs only then
+    big = (65536, 32, 0, 4096)                  # needs more scratch than the fixed array holds
+    assert lib.moe_dispatch_noalloc(N, *big, N, N, N, N) == 1
+    assert "null" in eb.last_error() and "moe_dispatch_noalloc" in eb.last_error()
+    assert lib.moe_dispatch_noalloc(a, 65536, 32, -1, 4096, a, a, a, N) == 1
+    assert lib.moe_dispatch_noalloc(odd, *big, a, a, a, N) == 1
+    assert "aligned" in eb.last_error()
+    assert lib.moe_dispatch_noalloc(a, 4, 8, 0, 0, a, a, a, N) == 2
+    assert lib.moe_dispatch_noalloc(a, *big, a, a, a, N) == 2
+    assert "scratch" in eb.last_error()
 
 
 def test_router_projection_arguments_checked_before_launch():

@@ -86,11 +86,12 @@ def test_cluster_combine_join(cuda_dev, T, H, k):
     torch.cuda.synchronize()
     branch_o = oracle_combine(case, synth.host(case.comb_wt))
     assert np.array_equal(synth.host(out), branch_o)
-    r_o, p_o = oracle.join(synth.host(case.residual), branch_o, synth.host(case.gain), case.alpha,
-                           case.beta, case.eps, synth.host(case.next_w), case.next_gc, case.eps)
+    r_o, p_o, n_o = oracle.join(synth.host(case.residual), branch_o, synth.host(case.gain), case.alpha,
+                                case.beta, case.eps, synth.host(case.next_w), case.next_gc, case.eps,
+                                return_normed=True)
     assert np.array_equal(synth.host(r).view(np.uint32), r_o.view(np.uint32))
     assert np.array_equal(synth.host(p), p_o)
-    check_join_outputs(synth.host(r), synth.host(p), r_o, p_o, case.beta)
+    check_join_outputs(synth.host(r), synth.host(p), r_o, p_o, n_o, case.beta)
 
 
 @pytest.mark.parametrize("H", [1024, 2688, 8192])

@@ -78,9 +78,9 @@ def test_random_shapes_match_the_oracle(cuda_dev, kind, seed):
     branch_o = oracle.combine(synth.host(case.expert_buf)[G:], case.R, synth.host(case.row_idx), w_o,
                               synth.host(case.post_w), case.post_gc, case.eps)
     assert bf16_ulp_diff(synth.host(out), branch_o).max() <= 1, shape
-    r_o, p_o2 = oracle.join(synth.host(case.residual), branch_o, synth.host(case.gain), case.alpha, case.beta,
-                            case.eps, synth.host(case.next_w), case.next_gc, case.eps)
-    check_join_outputs(synth.host(r), synth.host(p), r_o, p_o2, case.beta)
+    r_o, p_o2, n_o = oracle.join(synth.host(case.residual), branch_o, synth.host(case.gain), case.alpha, case.beta,
+                                 case.eps, synth.host(case.next_w), case.next_gc, case.eps, return_normed=True)
+    check_join_outputs(synth.host(r), synth.host(p), r_o, p_o2, n_o, case.beta)
 
     offs_o, row_idx_o, row_token_o = oracle.dispatch(synth.host(ids), 0, E)
     assert np.array_equal(synth.host(offs), offs_o), shape

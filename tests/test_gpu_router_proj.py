@@ -133,3 +133,30 @@ def test_router_weight_prepare_parts(cuda_dev):
     assert np.array_equal(got[0], b1) and np.array_equal(got[1], b2) and np.array_equal(got[2], b3)
     parts = sum(((got[p].astype(np.uint32) << 16).view(np.float32).astype(np.float64)) for p in range(3))
     assert np.all(np.abs(parts - wn.astype(np.float64)) <= 2.0 ** -27 * np.abs(wn.astype(np.float64)))
+
+
+def _experts_per_cta(T, E, H, sms):
+    """The tile the launch picks: 32 experts per CTA when E allows it and the
+    16-expert grid would take more than one wave at two CTAs per SM."""
+    ctas16 = (E // 16) * _chunks(H) * ((T + 127) // 128)
+    return 32 if E % 32 == 0 and ctas16 > 2 * sms else 16
+
+
+@pytest.mark.parametrize("T_small,T_big,H,E", [(128, 512, 8192, 256),     # C = 8
+                                               (100, 700, 64, 1024),      # C = 1, partial last tile
+                                               (60, 300, 128, 1024),      # C = 2
+                                               (90, 300, 256, 512)])      # C = 4
+def test_router_logits_equal_across_tile_widths(cuda_dev, T_small, T_big, H, E):
+    """The rows a small batch shares with a larger one come out bit-identical
+    whether the launch takes 16 or 32 experts per CTA (every output element is
+    summed in the same order either way)."""
+    sms = torch.cuda.get_device_properties(cuda_dev).multi_processor_count
+    assert _experts_per_cta(T_small, E, H, sms) == 16 and _experts_per_cta(T_big, E, H, sms) == 32
+    x, w = _inputs(T_big, H, E, seed=T_big + H + E)
+    w3 = eb.router_weight_prepare(w.to(cuda_dev))
+    xd = x.to(cuda_dev)
+    small = eb.router_logits(xd[:T_small].contiguous(), w3, 0.37)
+    big = eb.router_logits(xd, w3, 0.37)
+    torch.cuda.synchronize()
+    assert torch.equal(small, big[:T_small])
+    _check(x, w, 0.37, cuda_dev)

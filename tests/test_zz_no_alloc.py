@@ -6,8 +6,9 @@ instead of a caller workspace.
 
 Called through the C ABI (ctypes on the loaded library) with preallocated
 outputs, two calls in a row on different inputs, each compared with the
-workspace entry point moe_dispatch on the same ids.  The dispatch is integer
-work, so the comparison is exact.  This file is collected last on purpose.
+workspace entry point moe_dispatch on the same ids and with the CPU oracle's
+counting sort.  The dispatch is integer work, so the comparison is exact.
+This file is collected last on purpose.
 """
 import ctypes
 
@@ -16,6 +17,7 @@ import pytest
 import torch
 
 import expert_combine_b200 as eb
+import oracle
 from expert_combine_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -52,6 +54,8 @@ def test_noalloc_dispatch_equals_workspace_dispatch(cuda_dev, T, k, E):
         torch.cuda.synchronize()
         for g, w in zip(got, want):
             assert np.array_equal(synth.host(g), synth.host(w))
+        for g, o in zip(got, oracle.dispatch(synth.host(ids), 0, E)):
+            assert np.array_equal(synth.host(g).reshape(o.shape), o)
     assert eb.device_status() == 0
 
 
