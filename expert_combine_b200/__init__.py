@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     FAR_MAX_WORLD,
     IPC_HANDLE_BYTES,
     MoEBoundaryError,
+    ROUTE_FAST_SIGMOID_BOUND,
     STAGE_COMBINE,
     STAGE_COMBINE_JOIN,
     STAGE_DISPATCH,
@@ -42,6 +43,7 @@ from ._lib import (  # noqa: F401
     moe_dispatch,
     moe_dispatch_noalloc,
     moe_route,
+    moe_route_check_fast_sigmoid,
     moe_route_norm_quant,
     norm_quant_nvfp4,
     residual_join,

@@ -102,6 +102,7 @@ def load() -> ctypes.CDLL:
             P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
             sigs = {
                 "moe_route": [P, P, P, i32, i32, i32, P, P, P],
+                "moe_route_check_fast_sigmoid": [P, P],
                 "norm_quant_nvfp4": [P, i32, i32, i32, P, f32, f32, P, P, P, P],
                 "expert_combine": [P, i64, i32, P, P, i32, i32, P, f32, f32, P, P],
                 "residual_join": [P, P, P, f32, f32, f32, P, f32, f32, P, i32, i32, P],
@@ -199,6 +200,21 @@ def moe_route(logits: torch.Tensor, bias: torch.Tensor, token_mask: torch.Tensor
     _check("moe_route", load().moe_route(_ptr(logits), _ptr(bias), _ptr(token_mask), T, E, k,
                                          _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
     return topk_ids, topk_weights
+
+
+@_traced
+def moe_route_check_fast_sigmoid(stream=None) -> float:
+    """Largest |fast - exact| sigmoid over every binary32 input, measured on the
+    device (the bound moe_route's shortlist relies on); synchronises."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = torch.empty(1, dtype=torch.float32, device=dev)
+    _check("moe_route_check_fast_sigmoid", load().moe_route_check_fast_sigmoid(_ptr(out), _stream(stream)))
+    torch.cuda.synchronize(dev)
+    return float(out.item())
+
+
+# The bound moe_route's shortlist assumes (MB_ROUTE_FAST_SIGMOID_BOUND).
+ROUTE_FAST_SIGMOID_BOUND = 2.0 ** -21
 
 
 @_traced

@@ -114,6 +114,14 @@ static int check_route(const char* fn, const float* logits, const float* bias, c
     return MB_OK;
 }
 
+int moe_route_check_fast_sigmoid(float* max_err, void* stream) {
+    const char* fn = "moe_route_check_fast_sigmoid";
+    if (!max_err) return fail(MB_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if ((reinterpret_cast<uintptr_t>(max_err) & 3u) != 0)
+        return fail(MB_ERR_INVALID_ARG, "%s: max_err must be 4-byte aligned", fn);
+    return cuda_status(launch_fast_sigmoid_check(max_err, static_cast<cudaStream_t>(stream)), fn);
+}
+
 static int check_norm_quant(const char* fn, const uint16_t* x, int M, int H, int tp, const uint16_t* norm_w,
                             const float* global_scale, uint8_t* packed, uint8_t* sf) {
     if (M < 0 || H < 0 || tp < 0) return fail(MB_ERR_INVALID_ARG, "%s: negative size", fn);

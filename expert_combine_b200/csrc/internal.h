@@ -13,6 +13,8 @@ struct DeviceInfo {
 };
 const DeviceInfo& device_info();   // current device, cached per device
 
+// The exhaustive check of the router's fast sigmoid against the exact one.
+cudaError_t launch_fast_sigmoid_check(float* max_err, cudaStream_t s);
 cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                          int k, int32_t* ids, float* weights, cudaStream_t s);
 

@@ -9,22 +9,24 @@
 //   w_j   = s_{pick j} / (s_{pick 0} + ... + s_{pick k-1})   summed in pick order
 // and for an invalid token ids = -1, weights = 0 without reading its logits.
 //
-// Selection: every lane reads E/32 scores with 128-bit loads and turns each
-// into a 32-bit order-preserving key; k merge rounds then emit the picks in
-// order, each a warp max (redux.sync) over the lanes' current bests with the
-// lowest expert id winning among equal keys (a warp min over the tied
-// lanes).  For E <= 512 a lane keeps its best and second-best remaining
-// scores, promotes the second when its best is picked and rescans its <= 16
-// scores only when picked again before a rescan; beyond that it keeps a
-// sorted list of its best k.  Nothing is staged in
-// shared or global scratch memory.
+// Selection (route.cuh): a shortlist from a fast sigmoid with a bounded
+// error, then the exact sigmoid and an exact ranking of the shortlisted
+// experts only.  For E <= 512 a lane holds its E/32 logits in registers; for
+// larger E the approximate keys of the token go through one shared-memory row
+// per warp.  When the shortlist overflows (massive exact ties), the token
+// takes the exact merge rounds: k warp maxima (redux.sync) over the lanes'
+// best keys, the lowest expert id winning among equal keys.  Nothing is
+// staged in global scratch memory.
 #include "internal.h"
 #include "route.cuh"
 
 namespace mb {
 
-// MODE > 0: the small path with EPL = MODE scores per lane; MODE < 0: the
-// list path with L = -MODE entries.
+// MODE > 0: E <= 32 MODE, EPL = MODE logits per lane in registers (exact
+// rounds up to 8 per lane, the shortlist at 16); MODE < 0:
+// larger E, each lane keeping a sorted list of its L = -MODE best exact
+// scores (the router beside the norm-quant, which has no shared memory to
+// spare).
 //
 // BESIDE: launched right after the norm-quant kernel of the same tokens, to
 // run in the registers and warp slots that kernel leaves free on every SM.
@@ -34,8 +36,10 @@ namespace mb {
 // readers of ids / weights are done), and waits for it at the end, so that
 // the router finishes after the norm-quant and the kernels after it may rely
 // on both.
+// (the shortlist instantiation is held to four CTAs' registers per SM: more
+// warps hide its dependent chains; measured 115 -> 109 us at 65536 x 512, k = 22)
 template <int MODE, bool BESIDE>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256, (MODE > 8 && !BESIDE) ? 4 : 1) route_kernel(const float* __restrict__ logits,
                                                     const float* __restrict__ bias,
                                                     const uint8_t* __restrict__ mask, int T, int E,
                                                     int k, int32_t* __restrict__ ids,
@@ -48,9 +52,11 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     const bool vec = (E & 3) == 0;
 
     // one token per warp iteration: each token's selection is one dependent
-    // chain of warp reductions, and more warps with one chain each measured
-    // faster than fewer warps interleaving two
-    if constexpr (MODE > 0) {
+    // chain, and more warps with one chain each measured faster than fewer
+    // warps interleaving two
+    if constexpr (MODE > 8) {
+        route_shortlist_tokens<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
+    } else if constexpr (MODE > 0) {
         route_singles<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
     } else {
         for (int t = warp; t < T; t += nwarps) {
@@ -70,6 +76,25 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
         }
     }
     if constexpr (BESIDE) griddep_wait();
+}
+
+// E > 512 on its own: the shortlist over approximate keys staged in one
+// shared-memory row per warp (kRouteWideWarps warps per CTA).
+constexpr int kRouteWideWarps = 4;
+
+__global__ void __launch_bounds__(32 * kRouteWideWarps) route_wide_kernel(const float* __restrict__ logits,
+                                                                          const float* __restrict__ bias,
+                                                                          const uint8_t* __restrict__ mask, int T,
+                                                                          int E, int k, int32_t* __restrict__ ids,
+                                                                          float* __restrict__ weights) {
+    extern __shared__ __align__(16) uint32_t route_keys[];
+    griddep_wait();
+    griddep_launch();
+    const int lane = threadIdx.x & 31;
+    const int warp = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+    uint32_t* keys = route_keys + static_cast<size_t>(threadIdx.x >> 5) * 128 * ((E + 127) >> 7);
+    route_shortlist_tokens<0>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane, keys);
 }
 
 namespace {
@@ -95,12 +120,53 @@ cudaError_t launch_route_cfg(const float* logits, const float* bias, const uint8
     if (epl <= 4) return cudaLaunchKernelEx(&cfg, route_kernel<4, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
     if (epl <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<8, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
     if (epl <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
+    if constexpr (!BESIDE) {
+        // the shortlist with its keys in shared memory
+        const size_t smem = static_cast<size_t>(kRouteWideWarps) * 128 * ((E + 127) / 128) * sizeof(uint32_t);
+        cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(route_wide_kernel),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_wide_kernel, 32 * kRouteWideWarps, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        int g = (T + kRouteWideWarps - 1) / kRouteWideWarps;
+        if (g > device_info().sm_count * per_sm) g = device_info().sm_count * per_sm;
+        cfg.gridDim = dim3(g);
+        cfg.blockDim = dim3(32 * kRouteWideWarps);
+        cfg.dynamicSmemBytes = smem;
+        return cudaLaunchKernelEx(&cfg, route_wide_kernel, logits, bias, mask, T, E, k, ids, weights);
+    }
     if (k <= 8) return cudaLaunchKernelEx(&cfg, route_kernel<-8, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
     if (k <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<-16, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
     return cudaLaunchKernelEx(&cfg, route_kernel<-32, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
 }
 
 }  // namespace
+
+// Every binary32 input once: the largest |sigmoid_fast(x) - sigmoid_fixed(x)|
+// (NaN inputs skipped), as the bits of a non-negative float, max-combined into
+// *err_bits (which starts at 0).
+__global__ void __launch_bounds__(256) fast_sigmoid_check_kernel(unsigned int* __restrict__ err_bits) {
+    const uint64_t n = 1ull << 32;
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * blockDim.x;
+    uint32_t worst = 0u;
+    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const float x = __uint_as_float(static_cast<uint32_t>(i));
+        if (x != x) continue;
+        const float d = fabsf(__fsub_rn(sigmoid_fast(x), sigmoid_fixed(x)));
+        worst = max(worst, (d == d) ? __float_as_uint(d) : 0x7F800000u);
+    }
+    worst = __reduce_max_sync(0xffffffffu, worst);
+    if ((threadIdx.x & 31) == 0) atomicMax(err_bits, worst);
+}
+
+cudaError_t launch_fast_sigmoid_check(float* max_err, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(max_err, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    fast_sigmoid_check_kernel<<<device_info().sm_count * 8, 256, 0, s>>>(reinterpret_cast<unsigned int*>(max_err));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_route(const float* logits, const float* bias, const uint8_t* mask, int T, int E,
                          int k, int32_t* ids, float* weights, cudaStream_t s) {

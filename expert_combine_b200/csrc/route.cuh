@@ -9,6 +9,17 @@
 //   picks = first k experts in the order (c descending, id ascending)
 //   w_j   = s_{pick j} / (s_{pick 0} + ... + s_{pick k-1})   summed in pick order
 // and for an invalid token ids = -1, weights = 0 without reading its logits.
+//
+// Selection takes two steps per token.  A shortlist from a fast sigmoid (the
+// hardware's approximate 2^x and reciprocal, within kSigFastErr of the exact
+// one): k rounds of one warp max over each lane's two best approximate scores
+// give a value tau that at least k experts reach, and only experts whose
+// approximate score lies within twice the error bound below tau can belong to
+// the exact top k (every other one is exactly below k others).  Those
+// candidates -- typically k or a few more -- get the exact sigmoid, move to
+// one lane each and are ranked by broadcast, with no dependent chain of warp
+// reductions.  When more than 32 remain (massive exact ties) the token takes
+// the exact merge rounds over all its experts instead.
 #pragma once
 
 #include "common.cuh"
@@ -196,6 +207,341 @@ __device__ __forceinline__ void route_write(const float* l, int k, int lane, uin
     }
 }
 
+// ---------------------------------------------------------------- shortlist and verify
+// Fast sigmoid for the shortlist: 1 / (1 + 2^(-x log2 e)) with the hardware's
+// approximate 2^x and reciprocal (flush-to-zero).  Over all 2^32 binary32
+// inputs it differs from sigmoid_fixed by at most 1.79e-7 (2^-22.4) on sm_100a;
+// moe_route_check_fast_sigmoid measures that on the device, and kSigFastErr
+// bounds it with a margin.
+constexpr float kSigFastErr = 0x1p-21f;
+constexpr float kInf = __builtin_huge_valf();
+
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    const float t = __fmul_rn(x, -1.4426950408889634f);
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(t));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(__fadd_rn(1.0f, e)));
+    return r;
+}
+
+// The number a key > 1 stands for (inverse of score_key).
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Twice an upper bound on |c_fast - c| over a token's experts, where
+// c = fl(s + b) and c_fast = fl(s_fast + b): the sigmoid's error plus one ulp
+// of the largest |s + b| <= max|b| + 2 (a half-ulp rounding on each side);
+// infinite when a bias is not finite.  bmax_bits: the bits of max |b|.
+__device__ __forceinline__ float shortlist_width(uint32_t bmax_bits) {
+    const float B = __fadd_ru(__uint_as_float(bmax_bits), 2.0f);
+    const uint32_t ex = (__float_as_uint(B) >> 23) & 0xFFu;
+    if (ex == 0xFFu) return kInf;
+    const float ulp_b = __uint_as_float((ex - 23u) << 23);
+    return __fmul_ru(2.0f, __fadd_ru(kSigFastErr, ulp_b));
+}
+
+// The window's floor: an expert whose fast score is below it scores exactly
+// below every expert whose fast score reached tau (the k-th round's maximum,
+// as a key), and at least k did.  Rounded down; -inf keeps every number.
+__device__ __forceinline__ float shortlist_floor(uint32_t tau, float width) {
+    if (!(width < kInf)) return -kInf;
+    return __fsub_rd(key_value(tau), width);
+}
+
+// k rounds of the warp's best offer over each lane's two best fast scores
+// (as keys): every lane holding the round's maximum gives it up, so each round
+// removes at least one expert scoring at least the final maximum, returned.
+__device__ __forceinline__ uint32_t shortlist_tau(float a1f, float a2f, int k) {
+    uint32_t a1 = score_key(a1f), a2 = score_key(a2f), tau = 0u;
+    for (int j = 0; j < k; ++j) {
+        tau = warp_max_u32(a1);
+        if (a1 == tau) {
+            a1 = a2;
+            a2 = 0u;
+        }
+    }
+    return tau;
+}
+
+// Running best two of a lane's fast scores (NaN counts as -inf here).
+__device__ __forceinline__ void top2_update(float v, float& a1, float& a2) {
+    v = fmaxf(v, -kInf);
+    a2 = fmaxf(a2, fminf(v, a1));
+    a1 = fmaxf(a1, v);
+}
+
+// Position of the n-th (from 0) set bit of m; m has more than n set bits.
+__device__ __forceinline__ int nth_set_bit(uint32_t m, int n) {
+    int pos = 0;
+#pragma unroll
+    for (int w = 16; w > 0; w >>= 1) {
+        const int c = __popc(m & ((1u << w) - 1u));
+        if (n >= c) {
+            n -= c;
+            m >>= w;
+            pos += w;
+        }
+    }
+    return pos;
+}
+
+// Rank a token's shortlisted experts exactly and write its picks.  Each lane
+// holds `cnt` of them; next_id() yields the lane's next expert id (cnt calls).
+// The ids move to one lane each, every lane computes its expert's exact
+// sigmoid and selection key at once, and the ranks come from broadcasts.
+// Returns false, writing nothing, when the warp holds more than 32 or fewer
+// than k shortlisted experts.
+template <class NextId>
+__device__ __forceinline__ bool shortlist_finish(int cnt, int lane, int k, NextId&& next_id,
+                                                 const float* __restrict__ row, const float* __restrict__ bias,
+                                                 int32_t* id_row, float* w_row) {
+    constexpr uint32_t kAll = 0xffffffffu;
+    int incl = cnt;                                  // inclusive prefix of the counts
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kAll, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const int nc = __shfl_sync(kAll, incl, 31);
+    if (nc > 32 || nc < k) return false;
+    // slot d (lane d < nc) takes id d - start of the lane whose slots begin at
+    // `start`, the highest slot start at or below d
+    const int off = incl - cnt;
+    const uint32_t starts = __reduce_or_sync(kAll, cnt > 0 ? (1u << off) : 0u);
+    const uint32_t holders = __ballot_sync(kAll, cnt > 0);
+    int src = lane, rd = -1;
+    if (lane < nc) {
+        const int start = 31 - __clz(starts & (0xffffffffu >> (31 - lane)));
+        src = nth_set_bit(holders, __popc(starts & ((1u << start) - 1u)));
+        rd = lane - start;
+    }
+    const int rounds = __reduce_max_sync(kAll, cnt);
+    uint32_t mid = 0u;
+    for (int r = 0; r < rounds; ++r) {
+        const uint32_t cid = (r < cnt) ? next_id() : 0u;
+        const uint32_t g = __shfl_sync(kAll, cid, src);
+        if (rd == r) mid = g;
+    }
+    uint32_t mkey = 0u;
+    float ms = 0.0f;
+    if (lane < nc) {
+        ms = sigmoid_fixed(__ldg(row + mid));
+        mkey = score_key(__fadd_rn(ms, __ldg(bias + mid)));
+    }
+    // rank in the order (key descending, id ascending); four candidates per
+    // step so that their broadcasts overlap
+    int rank = 0;
+    for (int i0 = 0; i0 < nc; i0 += 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q;
+            const uint32_t ki = __shfl_sync(kAll, mkey, i & 31);
+            const uint32_t ii = __shfl_sync(kAll, mid, i & 31);
+            rank += (i < nc && (ki > mkey || (ki == mkey && ii < mid))) ? 1 : 0;
+        }
+    }
+    const bool pick = lane < nc && rank < k;
+    float S = 0.0f;                                  // the picks' sigmoids, summed in pick order
+    for (int p0 = 0; p0 < k; p0 += 4) {
+        float v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t b = __ballot_sync(kAll, pick && rank == p0 + q);
+            v[q] = __shfl_sync(kAll, ms, (__ffs(b) - 1) & 31);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (p0 + q < k) S = __fadd_rn(S, v[q]);
+    }
+    if (pick) {
+        id_row[rank] = static_cast<int32_t>(mid);
+        w_row[rank] = __fdiv_rn(ms, S);
+    }
+    return true;
+}
+
+// One token with E <= 32 EPL: the lane's EPL fast scores in registers.
+// Returns false (nothing written) when the shortlist does not fit.
+template <int EPL>
+__device__ __forceinline__ bool route_token_shortlist(const float* __restrict__ row, const float* __restrict__ bias,
+                                                      int E, int k, int lane, bool vec, float width, int32_t* id_row,
+                                                      float* w_row) {
+    float av[EPL];
+    float a1 = -kInf, a2 = -kInf;
+    {
+        float lv[EPL], bv[EPL];
+        load_logits<EPL>(row, E, lane, vec, lv);
+        load_logits<EPL>(bias, E, lane, vec, bv);
+#pragma unroll
+        for (int p = 0; p < EPL; ++p) {
+            av[p] = lane_pos_id(p, lane) < static_cast<uint32_t>(E) ? __fadd_rn(sigmoid_fast(lv[p]), bv[p])
+                                                                    : __int_as_float(0x7fc00000);
+            top2_update(av[p], a1, a2);
+        }
+    }
+    const float lo = shortlist_floor(shortlist_tau(a1, a2, k), width);
+    uint32_t rem = 0u;
+#pragma unroll
+    for (int p = 0; p < EPL; ++p) rem |= (av[p] >= lo) ? (1u << p) : 0u;
+    const int cnt = __popc(rem);
+    auto next_id = [&]() {
+        const int p = __ffs(rem) - 1;
+        rem &= rem - 1u;
+        return lane_pos_id(p, lane);
+    };
+    return shortlist_finish(cnt, lane, k, next_id, row, bias, id_row, w_row);
+}
+
+// Large E (more than 16 experts per lane): the fast scores go through the
+// warp's shared-memory row `keys` of at least 128 ceil(E / 128) words; the
+// score of expert 128 c + 4 lane + i is word 128 c + 32 i + lane (each lane
+// touches only its own words).  A lane keeps up to kWideLaneCands shortlisted
+// experts; when one has more, or the warp more than 32, it returns false and
+// writes nothing.
+constexpr int kWideLaneCands = 8;
+
+__device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, const float* __restrict__ bias, int E,
+                                                 int k, int lane, bool vec, float width, uint32_t* keys,
+                                                 int32_t* id_row, float* w_row) {
+    const int nch = (E + 127) >> 7;
+    const float nan = __int_as_float(0x7fc00000);
+    float a1 = -kInf, a2 = -kInf;
+    for (int c0 = 0; c0 < nch; c0 += 4) {          // four chunks' loads in flight at a time
+        float4 v[4], b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e0 = 128 * (c0 + u) + 4 * lane;
+            if (vec && e0 + 3 < E) {
+                v[u] = ld_nc_f4(row + e0);
+                b[u] = __ldg(reinterpret_cast<const float4*>(bias + e0));
+            } else {
+                v[u].x = (e0 + 0 < E) ? __ldg(row + e0 + 0) : 0.0f;
+                v[u].y = (e0 + 1 < E) ? __ldg(row + e0 + 1) : 0.0f;
+                v[u].z = (e0 + 2 < E) ? __ldg(row + e0 + 2) : 0.0f;
+                v[u].w = (e0 + 3 < E) ? __ldg(row + e0 + 3) : 0.0f;
+                b[u].x = (e0 + 0 < E) ? __ldg(bias + e0 + 0) : 0.0f;
+                b[u].y = (e0 + 1 < E) ? __ldg(bias + e0 + 1) : 0.0f;
+                b[u].z = (e0 + 2 < E) ? __ldg(bias + e0 + 2) : 0.0f;
+                b[u].w = (e0 + 3 < E) ? __ldg(bias + e0 + 3) : 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u;
+            if (c < nch) {
+                const int e0 = 128 * c + 4 * lane;
+                const float lv4[4] = {v[u].x, v[u].y, v[u].z, v[u].w}, bv4[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float f = (e0 + i < E) ? __fadd_rn(sigmoid_fast(lv4[i]), bv4[i]) : nan;
+                    keys[128 * c + 32 * i + lane] = __float_as_uint(f);
+                    top2_update(f, a1, a2);
+                }
+            }
+        }
+    }
+    const float lo = shortlist_floor(shortlist_tau(a1, a2, k), width);
+    int cnt = 0;
+    uint32_t cand[kWideLaneCands];                    // shortlisted experts, newest first
+#pragma unroll
+    for (int i = 0; i < kWideLaneCands; ++i) cand[i] = 0u;
+    for (int c = 0; c < nch; ++c) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (__uint_as_float(keys[128 * c + 32 * i + lane]) >= lo) {
+#pragma unroll
+                for (int q = kWideLaneCands - 1; q > 0; --q) cand[q] = cand[q - 1];
+                cand[0] = static_cast<uint32_t>(128 * c + 4 * lane + i);
+                ++cnt;
+            }
+        }
+    }
+    int taken = 0;
+    auto next_id = [&]() {
+        const int q = cnt - 1 - taken;                // oldest first
+        ++taken;
+        uint32_t e = cand[0];
+#pragma unroll
+        for (int i = 1; i < kWideLaneCands; ++i) e = (q == i) ? cand[i] : e;
+        return e;
+    };
+    return shortlist_finish(cnt > kWideLaneCands ? 33 : cnt, lane, k, next_id, row, bias, id_row, w_row);
+}
+
+// Exact merge rounds for the large-E path when its shortlist does not fit:
+// the exact keys overwrite the warp's shared-memory row (same layout), each
+// lane tracks its best two remaining (key, position) and rescans its own words
+// once both are taken; k rounds as in select_small.  Sets the lane's pick
+// (lane j < k: pick j).
+__device__ __forceinline__ void select_wide_exact(const float* __restrict__ l, const float* __restrict__ bias, int E,
+                                                  int k, int lane, bool vec, uint32_t* keys, uint32_t& pick_id) {
+    const int nch = (E + 127) >> 7;
+    for (int c = 0; c < nch; ++c) {
+        const int e0 = 128 * c + 4 * lane;
+        float lv[4], bv[4];
+        if (vec && e0 + 3 < E) {
+            const float4 v = ld_nc_f4(l + e0), b = __ldg(reinterpret_cast<const float4*>(bias + e0));
+            lv[0] = v.x; lv[1] = v.y; lv[2] = v.z; lv[3] = v.w;
+            bv[0] = b.x; bv[1] = b.y; bv[2] = b.z; bv[3] = b.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                lv[i] = (e0 + i < E) ? __ldg(l + e0 + i) : 0.0f;
+                bv[i] = (e0 + i < E) ? __ldg(bias + e0 + i) : 0.0f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            keys[128 * c + 32 * i + lane] = (e0 + i < E) ? score_key(__fadd_rn(sigmoid_fixed(lv[i]), bv[i])) : 0u;
+    }
+    // position p = 4 c + i of this lane <-> expert 128 c + 4 lane + i <-> word 128 c + 32 i + lane
+    auto word = [&](int p) { return 128 * (p >> 2) + 32 * (p & 3) + lane; };
+    auto expert = [&](int p) { return static_cast<uint32_t>(128 * (p >> 2) + 4 * lane + (p & 3)); };
+    uint32_t k1 = 0u, k2 = 0u;
+    int p1 = 0, p2 = 0;
+    bool have2 = true;
+    auto scan = [&]() {
+        k1 = k2 = 0u;
+        p1 = p2 = 0;
+        for (int p = 0; p < 4 * nch; ++p) {
+            const uint32_t v = keys[word(p)];
+            if (v > k1) {
+                k2 = k1;
+                p2 = p1;
+                k1 = v;
+                p1 = p;
+            } else if (v > k2) {
+                k2 = v;
+                p2 = p;
+            }
+        }
+        have2 = true;
+    };
+    scan();
+    for (int j = 0; j < k; ++j) {
+        uint32_t key_j, id_j;
+        if (pick_round(k1, expert(p1), key_j, id_j)) {
+            keys[word(p1)] = 0u;                      // taken
+            if (have2) {
+                k1 = k2;
+                p1 = p2;
+                have2 = false;
+            } else {
+                scan();
+            }
+        }
+        if (lane == j) pick_id = id_j;
+    }
+}
+
+// The shortlist window of a call, from the biases in memory.
+__device__ __forceinline__ float bias_width(const float* bias, int E, int lane) {
+    uint32_t m = 0u;
+    for (int e = lane; e < E; e += 32) m = max(m, __float_as_uint(fabsf(__ldg(bias + e))));
+    return shortlist_width(warp_max_u32(m));
+}
+
 // Larger E: every lane keeps a sorted list of its L best (key, id); ids arrive
 // in ascending order, so inserting strictly below equal keys keeps ties in id
 // order.
@@ -266,11 +612,12 @@ __device__ __forceinline__ void route_token_list(const float* l, const float* bi
 }
 
 
-// One token per warp iteration (t, t + nwarps, ...) on the small path
-// (E <= 32 * MODE), for the router kernels and the router warps of the fused
-// norm-quant kernel: one selection chain at a time measured faster than two
-// interleaved (or than the next token's logits held in registers).  The next
-// token's mask byte is read at the end of each iteration.
+// One token per warp iteration (t, t + nwarps, ...) with the exact merge
+// rounds (E <= 32 MODE, MODE <= 8), for the router kernels and the router
+// warps of the fused norm-quant kernel: one selection chain at a time measured
+// faster than two interleaved (or than the next token's logits held in
+// registers), and at these sizes faster than the shortlist.  The next token's
+// mask byte is read at the end of each iteration.
 template <int MODE>
 __device__ __forceinline__ void route_singles(const float* __restrict__ logits, const float* __restrict__ bias,
                                               const uint8_t* __restrict__ mask, int T, int E, int k,
@@ -301,6 +648,65 @@ __device__ __forceinline__ void route_singles(const float* __restrict__ logits, 
         if (tn >= T) break;
         t = tn;
         valid = mask[t] != 0;
+    }
+}
+
+// Validity of this warp's tokens t0, t0 + nwarps, ..., 32 of them, one mask
+// byte per lane in one load (bit j: token t0 + j nwarps is valid).
+__device__ __forceinline__ uint32_t warp_token_mask(const uint8_t* __restrict__ mask, int T, int64_t t0, int nwarps,
+                                                    int lane) {
+    const int64_t t = t0 + static_cast<int64_t>(lane) * nwarps;
+    return __ballot_sync(0xffffffffu, t < T && mask[t] != 0);
+}
+
+// Bring a logits row (E floats) into L2 ahead of its use, 128 bytes a lane.
+__device__ __forceinline__ void prefetch_row_l2(const float* row, int E, int lane) {
+    for (int e = 32 * lane; e < E; e += 32 * 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + e));
+}
+
+// One token per warp iteration with the shortlist: MODE > 0, E <= 32 MODE
+// with the fast scores in registers; MODE == 0, larger E through the warp's
+// shared-memory row `keys`.  The mask bytes of 32 tokens come in one load and
+// the next valid token's logits are prefetched into L2 while this one is
+// selected.  A token whose shortlist does not fit takes the exact rounds.
+template <int MODE>
+__device__ __forceinline__ void route_shortlist_tokens(const float* __restrict__ logits,
+                                                       const float* __restrict__ bias,
+                                                       const uint8_t* __restrict__ mask, int T, int E, int k,
+                                                       int32_t* __restrict__ ids, float* __restrict__ weights,
+                                                       int warp, int nwarps, int lane, uint32_t* keys = nullptr) {
+    const bool vec = (E & 3) == 0;
+    if (warp >= T) return;
+    const float width = bias_width(bias, E, lane);
+    uint32_t vbits = 0u;
+    for (int64_t j = 0, t = warp; t < T; ++j, t += nwarps) {
+        if ((j & 31) == 0) vbits = warp_token_mask(mask, T, t, nwarps, lane);
+        const bool valid = (vbits >> (j & 31)) & 1u;
+        const float* row = logits + static_cast<size_t>(t) * E;
+        const int64_t tn = t + nwarps;
+        const bool next_valid = ((j & 31) != 31) ? ((vbits >> ((j + 1) & 31)) & 1u) : (tn < T);
+        if (next_valid && tn < T) prefetch_row_l2(logits + static_cast<size_t>(tn) * E, E, lane);
+        int32_t* id_row = ids + static_cast<size_t>(t) * k;
+        float* w_row = weights + static_cast<size_t>(t) * k;
+        if (!valid) {
+            if (lane < k) {
+                id_row[lane] = -1;
+                w_row[lane] = 0.0f;
+            }
+            continue;
+        }
+        uint32_t pick_id = 0u;
+        if constexpr (MODE > 0) {
+            if (route_token_shortlist<MODE>(row, bias, E, k, lane, vec, width, id_row, w_row)) continue;
+            float lv[MODE];
+            load_logits<MODE>(row, E, lane, vec, lv);
+            uint32_t pick_key = 0u;
+            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+        } else {
+            if (route_token_wide(row, bias, E, k, lane, vec, width, keys, id_row, w_row)) continue;
+            select_wide_exact(row, bias, E, k, lane, vec, keys, pick_id);
+        }
+        route_write(row, k, lane, pick_id, id_row, w_row);
     }
 }
 

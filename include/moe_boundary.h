@@ -73,9 +73,29 @@ enum {
  *   token_mask    [T] uint8 (required) topk_ids      [T, k] int32 (out)
  *   topk_weights  [T, k] FP32 (out)
  * Supported: 1 <= k <= 32, k <= E <= 4096.
+ *
+ * The kernels shortlist experts with a fast sigmoid whose error against the
+ * exact one is bounded by MB_ROUTE_FAST_SIGMOID_BOUND and decide among the
+ * shortlist with the exact sigmoid, so the results are those of the exact
+ * definition above (moe_route_check_fast_sigmoid re-measures the bound).
  */
+#define MB_ROUTE_FAST_SIGMOID_BOUND 4.76837158203125e-07f   /* 2^-21 */
 int moe_route(const float* logits, const float* bias, const uint8_t* token_mask, int T, int E,
               int k, int32_t* topk_ids, float* topk_weights, void* stream);
+
+/*
+ * moe_route_check_fast_sigmoid -- measure the router's fast-sigmoid bound.
+ *
+ * No counterpart on the reference pages: moe_route picks its candidates with
+ * an approximate sigmoid built from the GPU's approximate 2^x and reciprocal
+ * and is exact only while that approximation stays within
+ * MB_ROUTE_FAST_SIGMOID_BOUND of the exact sigmoid.  This call evaluates both
+ * on the device for every binary32 input (NaNs skipped) and writes the largest
+ * absolute difference to *max_err (a device float the caller owns; set to 0
+ * first, then max-combined by the kernel).  Enqueued on `stream`; read
+ * *max_err after synchronising.  Takes about a millisecond on a B200.
+ */
+int moe_route_check_fast_sigmoid(float* max_err, void* stream);
 
 /*
  * norm_quant_nvfp4 -- pre-expert RMSNorm fused with NVFP4 quantisation.

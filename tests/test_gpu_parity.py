@@ -92,7 +92,7 @@ def test_route_norm_quant_kernel_count(cuda_dev):
 def test_route_integer_logits_many_ties(cuda_dev):
     g = torch.Generator(device=cuda_dev)
     g.manual_seed(5)
-    for E, k in ((16, 5), (64, 8), (256, 8)):
+    for E, k in ((16, 5), (64, 8), (256, 8), (1024, 8), (2560, 22)):
         case = synth.make_case("tiny", device=cuda_dev, T=64, E=E, k=k, H=64)
         case.logits.copy_(torch.randint(-2, 3, case.logits.shape, generator=g, device=cuda_dev))
         vals = torch.tensor([0.0, 0.125, -0.125], device=cuda_dev)
@@ -313,3 +313,48 @@ def test_joint_pre_expert_steps_feed_the_combine(cuda_dev, T, H):
         ids_o, w_o = oracle.route(synth.host(lg), synth.host(case.bias), synth.host(case.mask), k)
         assert bf16_ulp_diff(synth.host(out), oracle_combine(case, w_o)).max() <= 1
     assert eb.device_status() == 0
+
+
+def test_fast_sigmoid_bound_holds_for_every_input(cuda_dev):
+    """The router shortlists with a fast sigmoid and is exact only while that
+    stays within its stated bound of the exact sigmoid: measured here over
+    every binary32 input on this device."""
+    err = eb.moe_route_check_fast_sigmoid()
+    assert 0.0 < err <= eb.ROUTE_FAST_SIGMOID_BOUND, err
+
+
+@pytest.mark.parametrize("E,k", [(256, 8), (512, 22), (64, 32), (33, 32), (2560, 8), (4096, 32), (1030, 9)])
+def test_route_shortlist_overflow_takes_the_exact_rounds(cuda_dev, E, k):
+    """Logits far above the sigmoid's saturation give many exactly equal
+    scores, so more than 32 experts reach the shortlist window and the token
+    takes the exact rounds; ties still go to the lowest ids."""
+    case = synth.make_case("tiny", device=cuda_dev, T=40, E=E, k=k, H=64)
+    case.logits[:20] = 40.0                    # every sigmoid rounds to 1: all scores tie on bias
+    case.bias.zero_()
+    case.logits[20:, : E // 2] = 40.0           # half the experts tie
+    case.logits[case.mask == 0] = float("nan")
+    ids, _, _ = check_route(case)
+    got = synth.host(ids)
+    assert (got[0] == np.arange(k)).all()
+
+
+@pytest.mark.parametrize("E", [2560, 1024])
+def test_route_large_e_lane_holding_many_candidates(cuda_dev, E):
+    """Large E: experts 4, 8, 12 (one in each of lanes 1-3) score highest, and
+    ten experts of lane 0's slice (0-3, 128-131, 256, 257) come next, so close
+    together that all ten fall in the shortlist window -- more than one lane
+    keeps -- and the token takes the exact rounds (their sigmoids partly tie,
+    so the lowest ids win)."""
+    k = 5
+    case = synth.make_case("tiny", device=cuda_dev, T=8, E=E, k=k, H=64)
+    lane0 = [0, 1, 2, 3, 128, 129, 130, 131, 256, 257]
+    case.logits.fill_(-10.0)
+    for n, e in enumerate(lane0):
+        case.logits[:, e] = 5.0 + n * 1e-6
+    for n, e in enumerate((4, 8, 12)):
+        case.logits[:, e] = 6.0 + 0.1 * n
+    case.bias.zero_()
+    case.logits[case.mask == 0] = float("nan")
+    ids, _, _ = check_route(case)
+    got = synth.host(ids)[0].tolist()
+    assert got[:3] == [12, 8, 4] and set(got[3:]) <= set(lane0)
