@@ -14,12 +14,14 @@ Prints ONE JSON line (rank 0).  `value` is tokens/s over all ranks (weak
 scaling: every rank runs its own batch of 8192 tokens).  The per-step inputs
 (1.2 GB) are larger than the 126 MB L2, so no flush runs between steps.
 
-Timing: the K steps run back to back between two CUDA events on the launching
-stream (barrier + synchronize on both sides, max over ranks); no event sits
-between the kernels of the region, since one would keep the next kernel from
-launching early.  The per-stage times (`stages_ms`, and the combine's launch
-duration in `roofline`) come from a second region right after it: each stage
-alone, K back-to-back launches between two events.
+Timing: the K steps are captured once in a CUDA graph (the library's calls
+are capture-safe) and the timed region replays it between two CUDA events on
+the launching stream (barrier + synchronize on both sides, max over ranks), so
+the number is the GPU's and not the Python launch path's; no event sits between
+the kernels of the region, since one would keep the next kernel from launching
+early.  The same K steps launched one call at a time from Python are timed too
+(`stream_launch`).  The per-stage times (`stages_ms`, and the combine's launch
+duration in `roofline`) come from graphs of K launches of one stage.
 """
 from __future__ import annotations
 
@@ -315,23 +317,32 @@ def run_ours(args, info):
     torch.cuda.synchronize()
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
+    g_step = capture_graph(step, args.steps, dev)
+    g_pre = capture_graph(pre_expert, args.steps, dev)
+    g_cmb = capture_graph(combine, args.steps, dev)
+    g_step.replay()                                   # untimed: the graph's first launch
+    torch.cuda.synchronize()
 
     shard.barrier(info)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
         time.sleep(0.3)
         t_wall = time.perf_counter()
-        e0, e1 = timed(step, args.steps)
+        e0, e1 = timed(g_step.replay, 1)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     shard.barrier(info)
     step_ms = e0.elapsed_time(e1)
-    # each stage alone, back to back, for the per-kernel launch durations
-    pre_ev = timed(pre_expert, args.steps)
-    cmb_ev = timed(combine, args.steps)
+    # each stage alone, K launches in one graph, for the per-kernel launch durations
+    pre_ev = timed(g_pre.replay, 1)
+    cmb_ev = timed(g_cmb.replay, 1)
+    # the same steps launched one call at a time from Python
+    sl_ev = timed(step, args.steps)
     torch.cuda.synchronize()
     stage_ms = [pre_ev[0].elapsed_time(pre_ev[1]) / args.steps,
                 cmb_ev[0].elapsed_time(cmb_ev[1]) / args.steps]
+    stream_launch_ms = sl_ev[0].elapsed_time(sl_ev[1]) / args.steps
+    del g_step, g_pre, g_cmb
     combine_ms = stage_ms[1]
     step_ms_max = shard.max_over_ranks(step_ms, info)
     ms_per_step = step_ms_max / args.steps
@@ -390,7 +401,11 @@ def run_ours(args, info):
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},
             "stages_ms": {"route_norm_quant": stage_ms[0], "combine": stage_ms[1],
-                          "how": "each stage alone, K back-to-back launches between two events"},
+                          "how": "each stage alone, K launches in one CUDA graph, replayed between two events"},
+            "stream_launch": {"ms_per_step": stream_launch_ms,
+                              "tokens_per_s": shard.weak_scaling_throughput(T, stream_launch_ms, info),
+                              "how": "the same K steps launched call by call from Python between two events"},
+            "timing": "K steps captured in one CUDA graph, replayed between two events on the launching stream",
             "cpu_baseline": cpu,
             "e2e": e2e,
             "dispatch": disp,
@@ -410,6 +425,22 @@ def run_ours(args, info):
     if eb.device_status() != 0:
         raise RuntimeError("a kernel reported a wait timeout")
     return result
+
+
+def capture_graph(fn, n, dev):
+    """n calls of fn captured in one CUDA graph (after one call on a side
+    stream, which configures the kernels outside the capture)."""
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    return g
 
 
 def run_dispatch(eb, ids, E, dev, reps):
@@ -589,12 +620,15 @@ def run_leg(eb, name, dev, steps, warmup, peak):
         combine()
 
     def per_call_ms(fn, n):
+        g = capture_graph(fn, n, dev)
+        g.replay()
+        torch.cuda.synchronize()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for _ in range(n):
-            fn()
+        g.replay()
         t1.record(stream)
         torch.cuda.synchronize()
+        del g
         return t0.elapsed_time(t1) / n
 
     for _ in range(warmup):
@@ -628,7 +662,7 @@ def run_leg(eb, name, dev, steps, warmup, peak):
             "step_bytes_nominal": step_bytes, "bytes_per_token": b_route + b_nq + b_cmb,
             "step_gbs": step_gbs, "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS, "frac_of_measured": step_gbs / peak,
             "stages": stage_rep, "valid_slots": valid_slots,
-            "how": f"{steps} back-to-back steps between two events; each stage alone the same way",
+            "how": f"{steps} steps in one CUDA graph replayed between two events; each stage alone the same way",
             "gpu_launches_per_step": (eb.route_norm_quant_kernels(T, H, E, k, tp=case.tp)
                                       + (1 if not chained else 1 + (1 if T * k <= 4096 else
                                                                     (2 if T * k <= 32 * 4096 else 3))))}
