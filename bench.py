@@ -54,24 +54,27 @@ def bytes_per_token(H, E, k):
     return route, norm_quant, combine
 
 
-# DRAM traffic of one combine launch on this bench's default workload (8192
-# tokens): dram__bytes_read.sum + dram__bytes_write.sum, mean of the 6 launches
-# of one ncu launch-list capture.  It stands only while the kernel's sources
-# hash to `src` and the workload is unchanged; otherwise it is reported null.
-COMBINE_TRAFFIC = {"src": "307cae42447d4100", "tokens": 8192,
-                   "bytes": 1008076743 + 117870763}
+# DRAM traffic of one combine launch: dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture of a single combine_wide launch on
+# the prefill workload cut to 2048 tokens (profiles/combine_wide_prefill_T2048_
+# H8192_traffic.md), scaled to a launch of this bench by the algorithmic bytes
+# (the reads equal the algorithmic reads there, so the traffic grows with the
+# rows read).  It stands only while the kernel's sources hash to `src`;
+# otherwise it is reported null.
+COMBINE_TRAFFIC = {"src": "307cae42447d4100", "tokens": 2048, "bytes": 251303168 + 20315904,
+                   "algorithmic_bytes": 284786688}
 COMBINE_SOURCES = ("combine.cu", "ring.cuh", "common.cuh")
 
 
-def combine_traffic(T):
+def combine_traffic(algorithmic_bytes):
     import hashlib
     h = hashlib.sha256()
     for name in COMBINE_SOURCES:
         with open(os.path.join(ROOT, "expert_combine_b200", "csrc", name), "rb") as f:
             h.update(f.read())
-    if h.hexdigest()[:16] != COMBINE_TRAFFIC["src"] or T != COMBINE_TRAFFIC["tokens"]:
+    if h.hexdigest()[:16] != COMBINE_TRAFFIC["src"]:
         return None
-    return COMBINE_TRAFFIC["bytes"]
+    return int(round(COMBINE_TRAFFIC["bytes"] * algorithmic_bytes / COMBINE_TRAFFIC["algorithmic_bytes"]))
 
 
 def measured_peaks():
@@ -396,7 +399,8 @@ def run_ours(args, info):
                     "frac_of_measured": step_bytes_nominal / (ms_per_step * 1e-3) / 1e9 / peak},
             "roofline": {"kernel": "combine", "bound": "hbm", "achieved": achieved_cmb,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved_cmb / peak, "traffic": combine_traffic(T),
+                         "frac": achieved_cmb / peak, "traffic": combine_traffic(cmb_bytes_net),
+                         "traffic_source": "ncu, one combine launch at 2048 tokens, scaled by algorithmic bytes",
                          "bytes_per_launch": cmb_bytes_net,
                          "bytes_per_launch_nominal": cmb_bytes_nominal,
                          "avg_launch_ms": combine_ms},

@@ -323,40 +323,39 @@ __device__ __forceinline__ bool shortlist_finish(int cnt, int lane, int k, NextI
         const uint32_t g = __shfl_sync(kAll, cid, src);
         if (rd == r) mid = g;
     }
-    uint32_t mkey = 0u;
+    // the order (key descending, id ascending) as one 64-bit number, larger first
+    uint64_t mine = 0u;                              // lanes without a candidate sort last
     float ms = 0.0f;
     if (lane < nc) {
         ms = sigmoid_fixed(__ldg(row + mid));
-        mkey = score_key(__fadd_rn(ms, __ldg(bias + mid)));
+        const uint32_t key = score_key(__fadd_rn(ms, __ldg(bias + mid)));
+        mine = (static_cast<uint64_t>(key) << 32) | static_cast<uint64_t>(~mid);
     }
-    // rank in the order (key descending, id ascending); four candidates per
-    // step so that their broadcasts overlap
+    // rank: how many candidates come first; eight per step so that their
+    // broadcasts overlap
     int rank = 0;
-    for (int i0 = 0; i0 < nc; i0 += 4) {
+    for (int i0 = 0; i0 < nc; i0 += 8) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int i = i0 + q;
-            const uint32_t ki = __shfl_sync(kAll, mkey, i & 31);
-            const uint32_t ii = __shfl_sync(kAll, mid, i & 31);
-            rank += (i < nc && (ki > mkey || (ki == mkey && ii < mid))) ? 1 : 0;
+        for (int q = 0; q < 8; ++q) {
+            const uint64_t other = __shfl_sync(kAll, mine, (i0 + q) & 31);
+            rank += (other > mine) ? 1 : 0;
         }
     }
-    const bool pick = lane < nc && rank < k;
-    float S = 0.0f;                                  // the picks' sigmoids, summed in pick order
-    for (int p0 = 0; p0 < k; p0 += 4) {
-        float v[4];
+    // lane p learns which lane holds rank p: bit b of that lane's index, for
+    // every rank at once, in one warp OR per bit
+    int from = 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t b = __ballot_sync(kAll, pick && rank == p0 + q);
-            v[q] = __shfl_sync(kAll, ms, (__ffs(b) - 1) & 31);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            if (p0 + q < k) S = __fadd_rn(S, v[q]);
+    for (int bit = 0; bit < 5; ++bit) {
+        const uint32_t m = __reduce_or_sync(kAll, (lane < nc && ((lane >> bit) & 1)) ? (1u << rank) : 0u);
+        from |= static_cast<int>((m >> lane) & 1u) << bit;
     }
-    if (pick) {
-        id_row[rank] = static_cast<int32_t>(mid);
-        w_row[rank] = __fdiv_rn(ms, S);
+    const float sp = __shfl_sync(kAll, ms, from);    // lane p < k: the sigmoid of pick p
+    const uint32_t idp = __shfl_sync(kAll, mid, from);
+    float S = 0.0f;                                  // summed in pick order
+    for (int p = 0; p < k; ++p) S = __fadd_rn(S, __shfl_sync(kAll, sp, p));
+    if (lane < k) {
+        id_row[lane] = static_cast<int32_t>(idp);
+        w_row[lane] = __fdiv_rn(sp, S);
     }
     return true;
 }
