@@ -323,7 +323,8 @@ def run_ours(args, info):
     g_step = capture_graph(step, args.steps, dev)
     g_pre = capture_graph(pre_expert, args.steps, dev)
     g_cmb = capture_graph(combine, args.steps, dev)
-    g_step.replay()                                   # untimed: the graph's first launch
+    for g in (g_step, g_pre, g_cmb):                  # untimed: each graph's first launch uploads it
+        g.replay()
     torch.cuda.synchronize()
 
     shard.barrier(info)
