@@ -204,7 +204,41 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         cur->ct = ct;
         cur->cj = cj;
     };
-    if (tid == 0) {
+    // one-warp teams run the cursor together: the cursor token's row indices
+    // sit one per lane, its valid slots not yet requested in a ballot mask,
+    // so a refill is a shuffle and one copy instead of the leader's walk
+    int wc_t = static_cast<int>(blockIdx.x) * NTEAM + team;      // cursor token
+    int32_t wc_r = -1;                                          // its row index in this lane's slot
+    uint32_t wc_mask = 0u;                                      // its valid slots still to request
+    int wc_slot = 0, wc_issued = 0, wc_consumed = 0;
+    auto warp_issue = [&]() {
+        while (wc_mask == 0u) {
+            wc_t += team_stride;
+            if (wc_t >= T) return;
+            wc_r = lane < k ? __ldg(a.row_idx + static_cast<size_t>(wc_t) * k + lane) : -1;
+            wc_mask = __ballot_sync(0xffffffffu, lane < k && slot_valid(wc_r, R));
+        }
+        const int j = __ffs(wc_mask) - 1;
+        wc_mask &= wc_mask - 1u;
+        const int32_t r = __shfl_sync(0xffffffffu, wc_r, j);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&tb[wc_slot], 2u * static_cast<uint32_t>(H));
+            uint8_t* dst = ring + static_cast<size_t>(wc_slot) * slot_bytes;
+            if constexpr (SWZ)
+                tma_load_2d(smem_addr(dst), &tmap, 0, r * (H / 64), &tb[wc_slot]);
+            else
+                bulk_g2s(dst, a.expert_out + static_cast<size_t>(r) * H, 2u * static_cast<uint32_t>(H), &tb[wc_slot]);
+        }
+        wc_issued += 1;
+        wc_slot = (wc_slot + 1 == nslot) ? 0 : wc_slot + 1;
+    };
+    if constexpr (TW == 1) {
+        if (wc_t < T) {
+            wc_r = lane < k ? __ldg(a.row_idx + static_cast<size_t>(wc_t) * k + lane) : -1;
+            wc_mask = __ballot_sync(0xffffffffu, lane < k && slot_valid(wc_r, R));
+            for (int i = 0; i < nslot; ++i) warp_issue();
+        }
+    } else if (tid == 0) {
         *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
         for (int i = 0; i < nslot; ++i) issue();
     }
@@ -285,7 +319,12 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 aborted = true;
                 break;
             }
-            if (tid == 0) {   // the whole team has read these slots: refill them
+            if constexpr (TW == 1) {   // the warp has read these slots: refill them
+                wc_consumed += two ? 2 : 1;
+                if (lane == 0) fence_proxy_async_smem();
+                warp_issue();
+                if (two) warp_issue();
+            } else if (tid == 0) {   // the whole team has read these slots: refill them
                 cur->consumed += two ? 2 : 1;
                 fence_proxy_async_smem();
                 issue();
@@ -336,9 +375,14 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
         if constexpr (JOIN) join_token32<TW>(brw, t, H, tid, nvalid, a.join, team_sum, pow2, rH);
     }
     // copies still in flight (only after an abort) land before the CTA exits
-    if (tid == 0)
+    if constexpr (TW == 1) {
+        if (lane == 0)
+            for (int f = wc_consumed; f < wc_issued; ++f)
+                mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+    } else if (tid == 0) {
         for (int f = cur->consumed; f < cur->issued; ++f)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+    }
 }
 
 // ---------------------------------------------------------------------------
