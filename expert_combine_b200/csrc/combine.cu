@@ -446,31 +446,35 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     int* abort_word = abort_all + 4 * team;
     float* part = part_all + team * 2 * TW;
 
-    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
-    auto issue = [&]() {
-        int ct = cur->ct, cj = cur->cj;
-        while (ct < T) {
-            const int32_t r = __ldg(a.row_idx + static_cast<size_t>(ct) * k + cj);
-            if (++cj == k) {
-                cj = 0;
-                ct += team_stride;
-                if (ct + team_stride < T)
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(a.row_idx + static_cast<size_t>(ct + team_stride) * k));
-            }
-            if (!slot_valid(r, R)) continue;
-            const int ws = cur->wslot;
-            mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
-            tma_load_2d(smem_addr(ring + static_cast<size_t>(ws) * slot_bytes), &tmap, 0, r * lines, &tb[ws]);
-            cur->issued += 1;
-            cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
-            break;
+    // warp 0 of the team runs the copy cursor together: the cursor token's
+    // row indices one per lane, its valid slots not yet requested in a ballot
+    // mask, so a refill is a shuffle and one copy (lane 0 issues it)
+    int wc_t = static_cast<int>(blockIdx.x) * NTEAM + team;      // cursor token
+    int32_t wc_r = -1;
+    uint32_t wc_mask = 0u;
+    int wc_slot = 0, wc_issued = 0, wc_consumed = 0;
+    auto warp_issue = [&]() {
+        while (wc_mask == 0u) {
+            wc_t += team_stride;
+            if (wc_t >= T) return;
+            wc_r = lane < k ? __ldg(a.row_idx + static_cast<size_t>(wc_t) * k + lane) : -1;
+            wc_mask = __ballot_sync(0xffffffffu, lane < k && slot_valid(wc_r, R));
         }
-        cur->ct = ct;
-        cur->cj = cj;
+        const int j = __ffs(wc_mask) - 1;
+        wc_mask &= wc_mask - 1u;
+        const int32_t r = __shfl_sync(0xffffffffu, wc_r, j);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&tb[wc_slot], 2u * static_cast<uint32_t>(H));
+            tma_load_2d(smem_addr(ring + static_cast<size_t>(wc_slot) * slot_bytes), &tmap, 0, r * lines,
+                        &tb[wc_slot]);
+        }
+        wc_issued += 1;
+        wc_slot = (wc_slot + 1 == nslot) ? 0 : wc_slot + 1;
     };
-    if (tid == 0) {
-        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
-        for (int i = 0; i < nslot; ++i) issue();
+    if (warp_in_team == 0 && wc_t < T) {
+        wc_r = lane < k ? __ldg(a.row_idx + static_cast<size_t>(wc_t) * k + lane) : -1;
+        wc_mask = __ballot_sync(0xffffffffu, lane < k && slot_valid(wc_r, R));
+        for (int i = 0; i < nslot; ++i) warp_issue();
     }
 
     const float fH = static_cast<float>(H);
@@ -536,10 +540,10 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 aborted = true;
                 break;
             }
-            if (tid == 0 && held) {   // every warp has finished pass 2 of the previous row
-                cur->consumed += 1;
-                fence_proxy_async_smem();
-                issue();
+            if (warp_in_team == 0 && held) {   // every warp has finished pass 2 of the previous row
+                wc_consumed += 1;
+                if (lane == 0) fence_proxy_async_smem();
+                warp_issue();
             }
             held = true;
             float pp[TW];
@@ -584,7 +588,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     }
     // copies still in flight land before the CTA exits
     if (tid == 0)
-        for (int f = cur->consumed; f < cur->issued; ++f)
+        for (int f = wc_consumed; f < wc_issued; ++f)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
 }
 
