@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     if constexpr (ROUTE) {
         constexpr int RW = kFusedRouterWarps;
         if (warp >= NTEAM * TW) {
-            route_singles<8>(ra.logits, ra.bias, ra.mask, a.M, ra.E, ra.k, ra.ids, ra.weights,
+            route_singles<8, false>(ra.logits, ra.bias, ra.mask, a.M, ra.E, ra.k, ra.ids, ra.weights,
                            static_cast<int>(blockIdx.x) * RW + (warp - NTEAM * TW),
                            static_cast<int>(gridDim.x) * RW, lane);
             return;

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256, (MODE > 8 && !BESIDE) ? 4 : 1) route_kern
     if constexpr (MODE > 8) {
         route_shortlist_tokens<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
     } else if constexpr (MODE > 0) {
-        route_singles<MODE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
+        route_singles<MODE, !BESIDE>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane);
     } else {
         for (int t = warp; t < T; t += nwarps) {
             int32_t* id_row = ids + static_cast<size_t>(t) * k;

@@ -611,13 +611,15 @@ __device__ __forceinline__ void route_token_list(const float* l, const float* bi
 }
 
 
-// One token per warp iteration (t, t + nwarps, ...) with the exact merge
-// rounds (E <= 32 MODE, MODE <= 8), for the router kernels and the router
-// warps of the fused norm-quant kernel: one selection chain at a time measured
-// faster than two interleaved (or than the next token's logits held in
-// registers), and at these sizes faster than the shortlist.  The next token's
-// mask byte is read at the end of each iteration.
-template <int MODE>
+// One token per warp iteration (t, t + nwarps, ...) for E <= 32 MODE (MODE
+// <= 8), the next token's mask byte read at the end of each iteration: one
+// selection chain at a time measured faster than two interleaved (or than the
+// next token's logits held in registers).  SHORTLIST: the shortlist selection
+// (the standalone router kernels, where it measured faster: 10.2 -> 8.6 us at
+// 8192 x 256); otherwise the exact merge rounds over the lane's registers (the
+// router warps inside the norm-quant kernel, whose row warps the shortlist's
+// shuffles slowed: 41.3 -> 44.3 us for the fused call).
+template <int MODE, bool SHORTLIST>
 __device__ __forceinline__ void route_singles(const float* __restrict__ logits, const float* __restrict__ bias,
                                               const uint8_t* __restrict__ mask, int T, int E, int k,
                                               int32_t* __restrict__ ids, float* __restrict__ weights, int warp,
@@ -626,27 +628,52 @@ __device__ __forceinline__ void route_singles(const float* __restrict__ logits, 
     int t = warp;
     if (t >= T) return;
     bool valid = mask[t] != 0;
-    float lv[MODE];
-#pragma unroll
-    for (int i = 0; i < MODE; ++i) lv[i] = 0.0f;
-    for (;;) {
-        const int tn = t + nwarps;
-        if (valid) load_logits<MODE>(logits + static_cast<size_t>(t) * E, E, lane, vec, lv);
-        int32_t* id_row = ids + static_cast<size_t>(t) * k;
-        float* w_row = weights + static_cast<size_t>(t) * k;
-        if (!valid) {
-            if (lane < k) {
-                id_row[lane] = -1;
-                w_row[lane] = 0.0f;
+    if constexpr (SHORTLIST) {
+        const float width = bias_width(bias, E, lane);
+        for (;;) {
+            const int tn = t + nwarps;
+            int32_t* id_row = ids + static_cast<size_t>(t) * k;
+            float* w_row = weights + static_cast<size_t>(t) * k;
+            const float* row = logits + static_cast<size_t>(t) * E;
+            if (!valid) {
+                if (lane < k) {
+                    id_row[lane] = -1;
+                    w_row[lane] = 0.0f;
+                }
+            } else if (!route_token_shortlist<MODE>(row, bias, E, k, lane, vec, width, id_row, w_row)) {
+                float lv[MODE];
+                load_logits<MODE>(row, E, lane, vec, lv);
+                uint32_t pick_key = 0u, pick_id = 0u;
+                select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+                route_write(row, k, lane, pick_id, id_row, w_row);
             }
-        } else {
-            uint32_t pick_key = 0u, pick_id = 0u;
-            select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
-            route_write(logits + static_cast<size_t>(t) * E, k, lane, pick_id, id_row, w_row);
+            if (tn >= T) break;
+            t = tn;
+            valid = mask[t] != 0;
         }
-        if (tn >= T) break;
-        t = tn;
-        valid = mask[t] != 0;
+    } else {
+        float lv[MODE];
+#pragma unroll
+        for (int i = 0; i < MODE; ++i) lv[i] = 0.0f;
+        for (;;) {
+            const int tn = t + nwarps;
+            if (valid) load_logits<MODE>(logits + static_cast<size_t>(t) * E, E, lane, vec, lv);
+            int32_t* id_row = ids + static_cast<size_t>(t) * k;
+            float* w_row = weights + static_cast<size_t>(t) * k;
+            if (!valid) {
+                if (lane < k) {
+                    id_row[lane] = -1;
+                    w_row[lane] = 0.0f;
+                }
+            } else {
+                uint32_t pick_key = 0u, pick_id = 0u;
+                select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
+                route_write(logits + static_cast<size_t>(t) * E, k, lane, pick_id, id_row, w_row);
+            }
+            if (tn >= T) break;
+            t = tn;
+            valid = mask[t] != 0;
+        }
     }
 }
 
