@@ -87,13 +87,13 @@ __global__ void __launch_bounds__(32 * kRouteWideWarps) route_wide_kernel(const 
                                                                           const uint8_t* __restrict__ mask, int T,
                                                                           int E, int k, int32_t* __restrict__ ids,
                                                                           float* __restrict__ weights) {
-    extern __shared__ __align__(16) uint32_t route_keys[];
+    extern __shared__ __align__(16) uint16_t route_keys[];
     griddep_wait();
     griddep_launch();
     const int lane = threadIdx.x & 31;
     const int warp = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
-    uint32_t* keys = route_keys + static_cast<size_t>(threadIdx.x >> 5) * 128 * ((E + 127) >> 7);
+    uint16_t* keys = route_keys + static_cast<size_t>(threadIdx.x >> 5) * 128 * ((E + 127) >> 7);
     route_shortlist_tokens<0>(logits, bias, mask, T, E, k, ids, weights, warp, nwarps, lane, keys);
 }
 
@@ -122,7 +122,7 @@ cudaError_t launch_route_cfg(const float* logits, const float* bias, const uint8
     if (epl <= 16) return cudaLaunchKernelEx(&cfg, route_kernel<16, BESIDE>, logits, bias, mask, T, E, k, ids, weights);
     if constexpr (!BESIDE) {
         // the shortlist with its keys in shared memory
-        const size_t smem = static_cast<size_t>(kRouteWideWarps) * 128 * ((E + 127) / 128) * sizeof(uint32_t);
+        const size_t smem = static_cast<size_t>(kRouteWideWarps) * 128 * ((E + 127) / 128) * sizeof(uint16_t);
         cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(route_wide_kernel),
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;

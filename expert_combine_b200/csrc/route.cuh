@@ -393,16 +393,45 @@ __device__ __forceinline__ bool route_token_shortlist(const float* __restrict__ 
 }
 
 // Large E (more than 16 experts per lane): the fast scores go through the
-// warp's shared-memory row `keys` of at least 128 ceil(E / 128) words; the
-// score of expert 128 c + 4 lane + i is word 128 c + 32 i + lane (each lane
-// touches only its own words).  A lane keeps up to kWideLaneCands shortlisted
-// experts; when one has more, or the warp more than 32, it returns false and
-// writes nothing.
+// warp's shared-memory row `keys` as FP16 (128 ceil(E / 128) halves, 2 bytes
+// each: half the space of FP32, so more warps fit per SM); the score of
+// expert e is half e, lane l handling experts 128 c + 4 l .. + 3 of each chunk
+// c (one 8-byte store or load per chunk, conflict-free).  The FP16 rounding
+// widens the window by `store_err` (half an FP16 ulp of the largest score), so
+// every expert whose fast score reaches the floor still does after storing.
+// A lane keeps up to kWideLaneCands shortlisted experts; when one has more,
+// or the warp more than 32, it returns false and writes nothing.
 constexpr int kWideLaneCands = 8;
 
+__device__ __forceinline__ uint2 pack_f16x4(float a, float b, float c, float d) {
+    uint2 r;
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r.x) : "f"(a), "f"(b));
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r.y) : "f"(c), "f"(d));
+    return r;
+}
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(f) : "r"(w));
+    return f;
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, hi;\n\t}" : "=f"(f) : "r"(w));
+    return f;
+}
+
+// Half an FP16 ulp of the largest |fast score| (at most max|b| + 2), or
+// infinity when FP16 cannot hold it (every expert is then shortlisted).
+__device__ __forceinline__ float f16_store_err(uint32_t bmax_bits) {
+    const float B = __fadd_ru(__uint_as_float(bmax_bits), 2.0f);
+    if (!(B < 32768.0f)) return kInf;
+    const uint32_t ex = (__float_as_uint(B) >> 23) & 0xFFu;    // B >= 2: ex >= 128
+    return __uint_as_float((ex - 11u) << 23);                  // 2^(e - 11) = ulp_f16(B) / 2
+}
+
 __device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, const float* __restrict__ bias, int E,
-                                                 int k, int lane, bool vec, float width, uint32_t* keys,
-                                                 int32_t* id_row, float* w_row) {
+                                                 int k, int lane, bool vec, float width, float store_err,
+                                                 uint16_t* keys, int32_t* id_row, float* w_row) {
     const int nch = (E + 127) >> 7;
     const float nan = __int_as_float(0x7fc00000);
     float a1 = -kInf, a2 = -kInf;
@@ -430,28 +459,33 @@ __device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, 
             const int c = c0 + u;
             if (c < nch) {
                 const int e0 = 128 * c + 4 * lane;
-                const float lv4[4] = {v[u].x, v[u].y, v[u].z, v[u].w}, bv4[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float f = (e0 + i < E) ? __fadd_rn(sigmoid_fast(lv4[i]), bv4[i]) : nan;
-                    keys[128 * c + 32 * i + lane] = __float_as_uint(f);
-                    top2_update(f, a1, a2);
-                }
+                const float f0 = (e0 + 0 < E) ? __fadd_rn(sigmoid_fast(v[u].x), b[u].x) : nan;
+                const float f1 = (e0 + 1 < E) ? __fadd_rn(sigmoid_fast(v[u].y), b[u].y) : nan;
+                const float f2 = (e0 + 2 < E) ? __fadd_rn(sigmoid_fast(v[u].z), b[u].z) : nan;
+                const float f3 = (e0 + 3 < E) ? __fadd_rn(sigmoid_fast(v[u].w), b[u].w) : nan;
+                *reinterpret_cast<uint2*>(keys + e0) = pack_f16x4(f0, f1, f2, f3);
+                top2_update(f0, a1, a2);
+                top2_update(f1, a1, a2);
+                top2_update(f2, a1, a2);
+                top2_update(f3, a1, a2);
             }
         }
     }
-    const float lo = shortlist_floor(shortlist_tau(a1, a2, k), width);
+    const float lo = __fsub_rd(shortlist_floor(shortlist_tau(a1, a2, k), width), store_err);
     int cnt = 0;
     uint32_t cand[kWideLaneCands];                    // shortlisted experts, newest first
 #pragma unroll
     for (int i = 0; i < kWideLaneCands; ++i) cand[i] = 0u;
     for (int c = 0; c < nch; ++c) {
+        const int e0 = 128 * c + 4 * lane;
+        const uint2 h = *reinterpret_cast<const uint2*>(keys + e0);
+        const float fv[4] = {f16_lo(h.x), f16_hi(h.x), f16_lo(h.y), f16_hi(h.y)};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if (__uint_as_float(keys[128 * c + 32 * i + lane]) >= lo) {
+            if (fv[i] >= lo) {                        // NaN (past E) never
 #pragma unroll
                 for (int q = kWideLaneCands - 1; q > 0; --q) cand[q] = cand[q - 1];
-                cand[0] = static_cast<uint32_t>(128 * c + 4 * lane + i);
+                cand[0] = static_cast<uint32_t>(e0 + i);
                 ++cnt;
             }
         }
@@ -468,43 +502,39 @@ __device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, 
     return shortlist_finish(cnt > kWideLaneCands ? 33 : cnt, lane, k, next_id, row, bias, id_row, w_row);
 }
 
-// Exact merge rounds for the large-E path when its shortlist does not fit:
-// the exact keys overwrite the warp's shared-memory row (same layout), each
-// lane tracks its best two remaining (key, position) and rescans its own words
-// once both are taken; k rounds as in select_small.  Sets the lane's pick
-// (lane j < k: pick j).
+// Exact merge rounds for the large-E path when its shortlist does not fit,
+// with no scratch: each lane tracks its best two remaining (key, position) of
+// its experts 128 c + 4 lane + i, recomputing their exact keys from memory
+// when it rescans (only after both were taken); taken positions are bits of
+// a 128-bit mask (E <= 4096: at most 128 positions a lane).  k rounds as in
+// select_small.  Sets the lane's pick (lane j < k: pick j).
 __device__ __forceinline__ void select_wide_exact(const float* __restrict__ l, const float* __restrict__ bias, int E,
-                                                  int k, int lane, bool vec, uint32_t* keys, uint32_t& pick_id) {
-    const int nch = (E + 127) >> 7;
-    for (int c = 0; c < nch; ++c) {
-        const int e0 = 128 * c + 4 * lane;
-        float lv[4], bv[4];
-        if (vec && e0 + 3 < E) {
-            const float4 v = ld_nc_f4(l + e0), b = __ldg(reinterpret_cast<const float4*>(bias + e0));
-            lv[0] = v.x; lv[1] = v.y; lv[2] = v.z; lv[3] = v.w;
-            bv[0] = b.x; bv[1] = b.y; bv[2] = b.z; bv[3] = b.w;
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                lv[i] = (e0 + i < E) ? __ldg(l + e0 + i) : 0.0f;
-                bv[i] = (e0 + i < E) ? __ldg(bias + e0 + i) : 0.0f;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            keys[128 * c + 32 * i + lane] = (e0 + i < E) ? score_key(__fadd_rn(sigmoid_fixed(lv[i]), bv[i])) : 0u;
-    }
-    // position p = 4 c + i of this lane <-> expert 128 c + 4 lane + i <-> word 128 c + 32 i + lane
-    auto word = [&](int p) { return 128 * (p >> 2) + 32 * (p & 3) + lane; };
+                                                  int k, int lane, uint32_t& pick_id) {
+    const int npos = 4 * ((E + 127) >> 7);
     auto expert = [&](int p) { return static_cast<uint32_t>(128 * (p >> 2) + 4 * lane + (p & 3)); };
+    uint32_t taken[4] = {0u, 0u, 0u, 0u};
+    auto is_taken = [&](int p) {
+        const uint32_t w = (p < 32) ? taken[0] : (p < 64) ? taken[1] : (p < 96) ? taken[2] : taken[3];
+        return ((w >> (p & 31)) & 1u) != 0u;
+    };
+    auto take = [&](int p) {
+        const uint32_t m = 1u << (p & 31);
+        if (p < 32) taken[0] |= m;
+        else if (p < 64) taken[1] |= m;
+        else if (p < 96) taken[2] |= m;
+        else taken[3] |= m;
+    };
     uint32_t k1 = 0u, k2 = 0u;
     int p1 = 0, p2 = 0;
     bool have2 = true;
     auto scan = [&]() {
         k1 = k2 = 0u;
         p1 = p2 = 0;
-        for (int p = 0; p < 4 * nch; ++p) {
-            const uint32_t v = keys[word(p)];
+        for (int p = 0; p < npos; ++p) {
+            const uint32_t e = expert(p);
+            const uint32_t v = (e < static_cast<uint32_t>(E) && !is_taken(p))
+                                   ? score_key(__fadd_rn(sigmoid_fixed(__ldg(l + e)), __ldg(bias + e)))
+                                   : 0u;
             if (v > k1) {
                 k2 = k1;
                 p2 = p1;
@@ -521,7 +551,7 @@ __device__ __forceinline__ void select_wide_exact(const float* __restrict__ l, c
     for (int j = 0; j < k; ++j) {
         uint32_t key_j, id_j;
         if (pick_round(k1, expert(p1), key_j, id_j)) {
-            keys[word(p1)] = 0u;                      // taken
+            take(p1);
             if (have2) {
                 k1 = k2;
                 p1 = p2;
@@ -534,11 +564,16 @@ __device__ __forceinline__ void select_wide_exact(const float* __restrict__ l, c
     }
 }
 
-// The shortlist window of a call, from the biases in memory.
-__device__ __forceinline__ float bias_width(const float* bias, int E, int lane) {
+// The bits of max |bias| over the call's experts (from memory).
+__device__ __forceinline__ uint32_t bias_max_bits(const float* bias, int E, int lane) {
     uint32_t m = 0u;
     for (int e = lane; e < E; e += 32) m = max(m, __float_as_uint(fabsf(__ldg(bias + e))));
-    return shortlist_width(warp_max_u32(m));
+    return warp_max_u32(m);
+}
+
+// The shortlist window of a call, from the biases in memory.
+__device__ __forceinline__ float bias_width(const float* bias, int E, int lane) {
+    return shortlist_width(bias_max_bits(bias, E, lane));
 }
 
 // Larger E: every lane keeps a sorted list of its L best (key, id); ids arrive
@@ -700,10 +735,12 @@ __device__ __forceinline__ void route_shortlist_tokens(const float* __restrict__
                                                        const float* __restrict__ bias,
                                                        const uint8_t* __restrict__ mask, int T, int E, int k,
                                                        int32_t* __restrict__ ids, float* __restrict__ weights,
-                                                       int warp, int nwarps, int lane, uint32_t* keys = nullptr) {
+                                                       int warp, int nwarps, int lane, uint16_t* keys = nullptr) {
     const bool vec = (E & 3) == 0;
     if (warp >= T) return;
-    const float width = bias_width(bias, E, lane);
+    const uint32_t bmax = bias_max_bits(bias, E, lane);
+    const float width = shortlist_width(bmax);
+    const float store_err = MODE > 0 ? 0.0f : f16_store_err(bmax);
     uint32_t vbits = 0u;
     for (int64_t j = 0, t = warp; t < T; ++j, t += nwarps) {
         if ((j & 31) == 0) vbits = warp_token_mask(mask, T, t, nwarps, lane);
@@ -729,8 +766,8 @@ __device__ __forceinline__ void route_shortlist_tokens(const float* __restrict__
             uint32_t pick_key = 0u;
             select_small<MODE>(lv, bias, E, k, lane, vec, pick_key, pick_id);
         } else {
-            if (route_token_wide(row, bias, E, k, lane, vec, width, keys, id_row, w_row)) continue;
-            select_wide_exact(row, bias, E, k, lane, vec, keys, pick_id);
+            if (route_token_wide(row, bias, E, k, lane, vec, width, store_err, keys, id_row, w_row)) continue;
+            select_wide_exact(row, bias, E, k, lane, pick_id);
         }
         route_write(row, k, lane, pick_id, id_row, w_row);
     }
