@@ -372,11 +372,19 @@ __device__ __forceinline__ bool route_token_shortlist(const float* __restrict__ 
         float lv[EPL], bv[EPL];
         load_logits<EPL>(row, E, lane, vec, lv);
         load_logits<EPL>(bias, E, lane, vec, bv);
+        if (E == 32 * EPL) {                         // every position holds an expert
 #pragma unroll
-        for (int p = 0; p < EPL; ++p) {
-            av[p] = lane_pos_id(p, lane) < static_cast<uint32_t>(E) ? __fadd_rn(sigmoid_fast(lv[p]), bv[p])
-                                                                    : __int_as_float(0x7fc00000);
-            top2_update(av[p], a1, a2);
+            for (int p = 0; p < EPL; ++p) {
+                av[p] = __fadd_rn(sigmoid_fast(lv[p]), bv[p]);
+                top2_update(av[p], a1, a2);
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < EPL; ++p) {
+                av[p] = lane_pos_id(p, lane) < static_cast<uint32_t>(E) ? __fadd_rn(sigmoid_fast(lv[p]), bv[p])
+                                                                        : __int_as_float(0x7fc00000);
+                top2_update(av[p], a1, a2);
+            }
         }
     }
     const float lo = shortlist_floor(shortlist_tau(a1, a2, k), width);
@@ -459,10 +467,18 @@ __device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, 
             const int c = c0 + u;
             if (c < nch) {
                 const int e0 = 128 * c + 4 * lane;
-                const float f0 = (e0 + 0 < E) ? __fadd_rn(sigmoid_fast(v[u].x), b[u].x) : nan;
-                const float f1 = (e0 + 1 < E) ? __fadd_rn(sigmoid_fast(v[u].y), b[u].y) : nan;
-                const float f2 = (e0 + 2 < E) ? __fadd_rn(sigmoid_fast(v[u].z), b[u].z) : nan;
-                const float f3 = (e0 + 3 < E) ? __fadd_rn(sigmoid_fast(v[u].w), b[u].w) : nan;
+                float f0, f1, f2, f3;
+                if (128 * (c + 1) <= E) {                // a full chunk (the same for the whole warp)
+                    f0 = __fadd_rn(sigmoid_fast(v[u].x), b[u].x);
+                    f1 = __fadd_rn(sigmoid_fast(v[u].y), b[u].y);
+                    f2 = __fadd_rn(sigmoid_fast(v[u].z), b[u].z);
+                    f3 = __fadd_rn(sigmoid_fast(v[u].w), b[u].w);
+                } else {
+                    f0 = (e0 + 0 < E) ? __fadd_rn(sigmoid_fast(v[u].x), b[u].x) : nan;
+                    f1 = (e0 + 1 < E) ? __fadd_rn(sigmoid_fast(v[u].y), b[u].y) : nan;
+                    f2 = (e0 + 2 < E) ? __fadd_rn(sigmoid_fast(v[u].z), b[u].z) : nan;
+                    f3 = (e0 + 3 < E) ? __fadd_rn(sigmoid_fast(v[u].w), b[u].w) : nan;
+                }
                 *reinterpret_cast<uint2*>(keys + e0) = pack_f16x4(f0, f1, f2, f3);
                 top2_update(f0, a1, a2);
                 top2_update(f1, a1, a2);
