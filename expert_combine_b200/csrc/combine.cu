@@ -308,12 +308,11 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                 for (int i = 0; i < 16; ++i) wv0[i] = wv1[i] = 0u;
             }
             bool abort;
-            float2 ss;
+            float ss;       // lane l: the sum of squares of the step's row l & 1
             if (two) {
-                ss = team_sum.sum2(row32_sumsq(wv0), row32_sumsq(wv1), !ok, abort);
+                ss = team_sum.sum2_lane(row32_sumsq(wv0), row32_sumsq(wv1), !ok, abort);
             } else {
-                ss.x = team_sum(row32_sumsq(wv0), !ok, abort);
-                ss.y = ss.x;
+                ss = team_sum(row32_sumsq(wv0), !ok, abort);
             }
             if (abort) {
                 aborted = true;
@@ -338,11 +337,14 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
                     phase ^= 1;
                 }
             }
-            const float inv0 = inv_rms_h(ss.x, fH, rH, pow2, a.eps);
+            // each lane forms the inverse RMS of its row l & 1 (one evaluation
+            // serves both rows); lanes 0 and 1 hand them out
+            const float inv_l = inv_rms_h(ss, fH, rH, pow2, a.eps);
+            const float inv0 = __shfl_sync(0xffffffffu, inv_l, 0);
             const float2 inv02 = make_float2(inv0, inv0);
             const float2 w02 = make_float2(w0, w0);
             if (two) {
-                const float inv1 = inv_rms_h(ss.y, fH, rH, pow2, a.eps);
+                const float inv1 = __shfl_sync(0xffffffffu, inv_l, 1);
                 const float2 inv12 = make_float2(inv1, inv1);
                 const float2 w12 = make_float2(w1, w1);
 #pragma unroll

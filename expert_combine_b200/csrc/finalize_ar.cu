@@ -213,13 +213,16 @@ __global__ void __launch_bounds__(NW * 32) finalize_ar_kernel(const FarArgs a) {
                 for (int i = 0; i < 16; ++i) x1[i] = 0u;
             }
             const float2 ss = cta_sum2<NW>(row32_sumsq(x0), row32_sumsq(x1), red);
-            const float inv0 = inv_rms_h(ss.x, fH, rH, pow2, a.eps);
+            // each lane forms the inverse RMS of row l & 1 of the step (one
+            // evaluation serves both rows); lanes 0 and 1 hand them out
+            const float inv_l = inv_rms_h((lane & 1) ? ss.y : ss.x, fH, rH, pow2, a.eps);
+            const float inv0 = __shfl_sync(0xffffffffu, inv_l, 0);
             const float2 inv02 = make_float2(inv0, inv0);
             const float2 w02 = make_float2(w0, w0);
 #pragma unroll
             for (int i = 0; i < 16; ++i) acc[i] = fma2(w02, far_norm_pair<GC0>(x0[i], wp[i], g[i], inv02), acc[i]);
             if (two) {
-                const float inv1 = inv_rms_h(ss.y, fH, rH, pow2, a.eps);
+                const float inv1 = __shfl_sync(0xffffffffu, inv_l, 1);
                 const float2 inv12 = make_float2(inv1, inv1);
                 const float2 w12 = make_float2(w1, w1);
 #pragma unroll

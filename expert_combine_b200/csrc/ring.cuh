@@ -165,6 +165,27 @@ struct TeamSum {
             return make_float2(tree_sum_array<TW>(p0), tree_sum_array<TW>(p1));
         }
     }
+
+    // Two independent sums; lane l receives the sum of v0 when l is even, of
+    // v1 when l is odd.  A one-warp team splits the butterfly's first level
+    // between the two sums (even lanes keep v0 and take the partner's v0, odd
+    // lanes the same for v1), so every later level moves one value instead of
+    // two; each sum still comes out of the balanced pairwise tree over lanes
+    // 0..31 in order.
+    __device__ __forceinline__ float sum2_lane(float v0, float v1, bool fail, bool& abort) {
+        if constexpr (TW == 1) {
+            const bool odd = (lane & 1) != 0;
+            float v = (odd ? v1 : v0) + __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+#pragma unroll
+            for (int off = 2; off < 32; off <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, off);
+            abort = __any_sync(0xffffffffu, fail);
+            __syncwarp();
+            return v;
+        } else {
+            const float2 s = sum2(v0, v1, fail, abort);
+            return (lane & 1) ? s.y : s.x;
+        }
+    }
 };
 
 // Reads this thread's 32 elements (16 words of two BF16) of a row slot.
