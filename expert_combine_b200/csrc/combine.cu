@@ -20,6 +20,7 @@
 // Fused after the combine, `branch` is the BF16 combine output.
 #include "internal.h"
 #include "ring.cuh"
+#include "tmem.cuh"
 #include "tmap.h"
 
 namespace mb {
@@ -395,9 +396,12 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // pass 1 forms the sum-of-squares partial (the team barrier then yields inv),
 // pass 2 re-reads the row, normalises it and accumulates; only the FP32
 // accumulator lives in registers.  A slot is handed back one row late (at the
-// barrier of the team's next row, when every warp has finished pass 2), and
-// the packed BF16 weights sit in a shared-memory table laid out so that both
-// the swizzled row lines and the table are read without bank conflicts.
+// barrier of the team's next row, when every warp has finished pass 2).  The
+// packed BF16 norm weights sit in tensor memory, not shared memory: lane l of
+// lane quadrant g holds the 32 weight words of line 32 (g % TW) + l (for
+// TW = 8, column block 1 holds the lines of warps 4..7 of a team), so pass 2
+// fetches them with tcgen05.ld and the shared-memory port carries only the
+// row copies and the two passes' reads of them.
 template <int TW, bool GC0>
 __global__ void __launch_bounds__(kConsumerThreads, 1)
     combine_wide_kernel(const __grid_constant__ CUtensorMap tmap, const CombineArgs a) {
@@ -410,7 +414,6 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int nslot = a.nslot;
     const int slot_bytes = slot_bytes_for(H);
     const WideLayout lay{NTEAM, nslot, slot_bytes, P};
-    uint4* wtab = reinterpret_cast<uint4*>(smem + lay.wtab_offset());
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
     float* part_all = reinterpret_cast<float*>(smem + lay.part_offset());
     int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
@@ -422,28 +425,78 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int tid = warp_in_team * 32 + lane;
     const int lines = H / 64;
     const bool has_line = tid < lines;
+    const bool warp_has_line = warp_in_team * 32 < lines;   // the same on every lane of the warp
+    // tensor-memory columns of one line's weights: 32 packed BF16 pairs, or
+    // with a gain centre the 64 FP32 gains gc + w (formed once here, the same
+    // single rounding as forming them per row)
+    constexpr uint32_t kLineCols = GC0 ? 32u : 64u;
+    constexpr int kColBlocks = TW > 4 ? 2 : 1;
+    constexpr uint32_t kWCols = kLineCols * kColBlocks;
+    __shared__ uint32_t s_tmem;
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, kWCols);
+        tmem_relinquish();
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);
         for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
         fence_mbar_init();
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     griddep_wait();     // row indices and weights may come from the previous kernel
     griddep_launch();
-    if (team == 0) {    // the weight table, chunk c of line t at [c][t]
+    if (warp < 4) {     // the weight table: quadrant `warp`, column block cb
+        const uint32_t tmem_base = s_tmem;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-            wtab[c * P + tid] = has_line ? *reinterpret_cast<const uint4*>(a.w + 64 * tid + 8 * c)
-                                         : make_uint4(0u, 0u, 0u, 0u);
+        for (int cb = 0; cb < kColBlocks; ++cb) {
+            const int line = ((warp % TW) + 4 * cb) * 32 + lane;
+            const uint32_t dst = tmem_base + ((32u * static_cast<uint32_t>(warp)) << 16) + kLineCols * cb;
+#pragma unroll
+            for (int h = 0; h < static_cast<int>(kLineCols / 32); ++h) {
+                uint32_t r[32];
+                if constexpr (GC0) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = line < lines ? *reinterpret_cast<const uint4*>(a.w + 64 * line + 8 * c)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                        r[4 * c] = v.x;
+                        r[4 * c + 1] = v.y;
+                        r[4 * c + 2] = v.z;
+                        r[4 * c + 3] = v.w;
+                    }
+                } else {   // elements 32 h .. 32 h + 31 of the line
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = line < lines
+                                            ? *reinterpret_cast<const uint4*>(a.w + 64 * line + 32 * h + 8 * c)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+                        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float2 f = unpack_bf16x2(ws[q]);
+                            r[8 * c + 2 * q] = __float_as_uint(line < lines ? __fadd_rn(a.gc, f.x) : 0.0f);
+                            r[8 * c + 2 * q + 1] = __float_as_uint(line < lines ? __fadd_rn(a.gc, f.y) : 0.0f);
+                        }
+                    }
+                }
+                tmem_st32(dst + 32u * static_cast<uint32_t>(h), r);
+            }
+        }
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    // this thread's line of weights: its warp's quadrant, its column block
+    const uint32_t wt_taddr = s_tmem + ((32u * static_cast<uint32_t>(warp & 3)) << 16) +
+                              kLineCols * static_cast<uint32_t>(warp_in_team >> 2);
 
     const int T = a.T, k = a.k;
     const int64_t R = a.R;
     const int team_stride = gridDim.x * NTEAM;
     uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
     const uint32_t ring_saddr = smem_addr(ring);
-    const uint32_t wtab_saddr = smem_addr(wtab);
     uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
     int* abort_word = abort_all + 4 * team;
     float* part = part_all + team * 2 * TW;
@@ -482,9 +535,9 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const float fH = static_cast<float>(H);
     const bool pow2 = (H & (H - 1)) == 0;
     const float rH = pow2 ? __frcp_rn(fH) : 0.0f;
-    const float2 gc2 = make_float2(a.gc, a.gc);
-    // swizzled position of chunk c of this thread's line (SWIZZLE_128B)
-    const uint32_t line_off = 128u * static_cast<uint32_t>(tid);
+    // this thread's line in a slot (line 0 for a thread past the row's end);
+    // chunk c of it sits at chunk c ^ sw (SWIZZLE_128B)
+    const uint32_t line_off = has_line ? 128u * static_cast<uint32_t>(tid) : 0u;
     const int sw = tid & 7;
 
     int t = blockIdx.x * NTEAM + team;
@@ -555,20 +608,30 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
             const float inv = inv_rms_h(tree_sum_array<TW>(pp), fH, rH, pow2, a.eps);
             const float2 inv2 = make_float2(inv, inv);
             const float2 w2 = make_float2(wj, wj);
-            // pass 2: normalise and accumulate
-            if (has_line) {
+            // pass 2: normalise and accumulate (every lane of a warp that holds
+            // a line reads the weight table; a lane past the row's end reads
+            // line 0 and its accumulator is never stored)
+            if (warp_has_line)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 x = lds128(sbase + 16u * static_cast<uint32_t>(c ^ sw));
-                    const uint4 wv = lds128(wtab_saddr + 16u * static_cast<uint32_t>(c * P + tid));
-                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-                    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+            for (int c = 0; c < 8; ++c) {
+                uint32_t ws[8];
+                if constexpr (GC0) {
+                    const uint4 wv = tmem_ld4_ro(wt_taddr + 4u * static_cast<uint32_t>(c));
+                    ws[0] = wv.x;
+                    ws[1] = wv.y;
+                    ws[2] = wv.z;
+                    ws[3] = wv.w;
+                } else {
+                    tmem_ld8_ro(wt_taddr + 8u * static_cast<uint32_t>(c), ws);
+                }
+                const uint4 x = lds128(sbase + 16u * static_cast<uint32_t>(c ^ sw));
+                const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float2 xg = GC0 ? mul_bf16x2_exact(xs[q], ws[q])
-                                              : mul2(unpack_bf16x2(xs[q]), add2(gc2, unpack_bf16x2(ws[q])));
-                        acc[4 * c + q] = fma2(w2, round_bf16_f2(mul2(xg, inv2)), acc[4 * c + q]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const float2 xg = GC0 ? mul_bf16x2_exact(xs[q], ws[q])
+                                          : mul2(unpack_bf16x2(xs[q]),
+                                                 make_float2(__uint_as_float(ws[2 * q]), __uint_as_float(ws[2 * q + 1])));
+                    acc[4 * c + q] = fma2(w2, round_bf16_f2(mul2(xg, inv2)), acc[4 * c + q]);
                 }
             }
             if (++slot == nslot) {
@@ -592,6 +655,12 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     if (tid == 0)
         for (int f = wc_consumed; f < wc_issued; ++f)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+    tc_fence_before();
+    __syncthreads();    // every warp's last weight-table read is done
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(s_tmem, kWCols);
+    }
 }
 
 // Standalone gated residual join: the branch comes from global memory.
