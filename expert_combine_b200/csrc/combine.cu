@@ -20,7 +20,6 @@
 // Fused after the combine, `branch` is the BF16 combine output.
 #include "internal.h"
 #include "ring.cuh"
-#include "tmem.cuh"
 #include "tmap.h"
 
 namespace mb {
@@ -426,15 +425,10 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int lines = H / 64;
     const bool has_line = tid < lines;
     const bool warp_has_line = warp_in_team * 32 < lines;   // the same on every lane of the warp
-    // tensor-memory columns of one line's weights: 32 packed BF16 pairs, or
-    // with a gain centre the 64 FP32 gains gc + w (formed once here, the same
-    // single rounding as forming them per row)
-    constexpr uint32_t kLineCols = GC0 ? 32u : 64u;
-    constexpr int kColBlocks = TW > 4 ? 2 : 1;
-    constexpr uint32_t kWCols = kLineCols * kColBlocks;
+    using WTab = WideWeightTable<TW, !GC0>;   // with a gain centre: the FP32 gains
     __shared__ uint32_t s_tmem;
     if (warp == 0) {
-        tmem_alloc(&s_tmem, kWCols);
+        tmem_alloc(&s_tmem, WTab::kCols);
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
@@ -447,50 +441,11 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     tc_fence_after();
     griddep_wait();     // row indices and weights may come from the previous kernel
     griddep_launch();
-    if (warp < 4) {     // the weight table: quadrant `warp`, column block cb
-        const uint32_t tmem_base = s_tmem;
-#pragma unroll
-        for (int cb = 0; cb < kColBlocks; ++cb) {
-            const int line = ((warp % TW) + 4 * cb) * 32 + lane;
-            const uint32_t dst = tmem_base + ((32u * static_cast<uint32_t>(warp)) << 16) + kLineCols * cb;
-#pragma unroll
-            for (int h = 0; h < static_cast<int>(kLineCols / 32); ++h) {
-                uint32_t r[32];
-                if constexpr (GC0) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = line < lines ? *reinterpret_cast<const uint4*>(a.w + 64 * line + 8 * c)
-                                                     : make_uint4(0u, 0u, 0u, 0u);
-                        r[4 * c] = v.x;
-                        r[4 * c + 1] = v.y;
-                        r[4 * c + 2] = v.z;
-                        r[4 * c + 3] = v.w;
-                    }
-                } else {   // elements 32 h .. 32 h + 31 of the line
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = line < lines
-                                            ? *reinterpret_cast<const uint4*>(a.w + 64 * line + 32 * h + 8 * c)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-                        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float2 f = unpack_bf16x2(ws[q]);
-                            r[8 * c + 2 * q] = __float_as_uint(line < lines ? __fadd_rn(a.gc, f.x) : 0.0f);
-                            r[8 * c + 2 * q + 1] = __float_as_uint(line < lines ? __fadd_rn(a.gc, f.y) : 0.0f);
-                        }
-                    }
-                }
-                tmem_st32(dst + 32u * static_cast<uint32_t>(h), r);
-            }
-        }
-    }
+    if (warp < 4) WTab::fill(s_tmem, warp, lane, a.w, a.gc, lines);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // this thread's line of weights: its warp's quadrant, its column block
-    const uint32_t wt_taddr = s_tmem + ((32u * static_cast<uint32_t>(warp & 3)) << 16) +
-                              kLineCols * static_cast<uint32_t>(warp_in_team >> 2);
+    const uint32_t wt_taddr = WTab::line_addr(s_tmem, warp, warp_in_team);
 
     const int T = a.T, k = a.k;
     const int64_t R = a.R;
@@ -659,7 +614,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     __syncthreads();    // every warp's last weight-table read is done
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(s_tmem, kWCols);
+        tmem_dealloc(s_tmem, WTab::kCols);
     }
 }
 

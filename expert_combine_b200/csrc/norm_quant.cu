@@ -44,6 +44,7 @@ struct FusedRouteArgs {
 // per SM sub-partition; at 896 threads the kernel fits in 72 registers a
 // thread without spilling.
 constexpr int kFusedRouterWarps = 12;
+constexpr int kTmemReleaseBar = 15;       // named barrier of the row warps at the end (teams use 1..8)
 // The router warps use the small selection path with 8 scores per lane.
 constexpr int kFusedRouteMaxExperts = 256;
 
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     const int nslot = a.nslot;
     const int slot_bytes = slot_bytes_for(H);
     const WideLayout lay{NTEAM, nslot, slot_bytes, P};
-    uint4* wtab = reinterpret_cast<uint4*>(smem + lay.wtab_offset());
+    uint4* wtab = reinterpret_cast<uint4*>(smem + lay.wtab_offset());   // used without the router warps
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
     float* part_all = reinterpret_cast<float*>(smem + lay.part_offset());
     int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
@@ -245,21 +246,41 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     const int tid = warp_in_team * 32 + lane;
     const int lines = H / 64;
     const bool has_line = tid < lines;
+    const bool warp_has_line = warp_in_team * 32 < lines;   // the same on every lane of the warp
+    // The packed BF16 norm weights: alone, the kernel reads them from a
+    // shared-memory table (chunk c of line t at [c][t]); with the router warps
+    // they sit in tensor memory instead and each block's eight words are
+    // fetched with tcgen05.ld, which leaves the shared-memory port to the rows
+    // (40.4 against 41.4 us for the fused call at 8192 x 8192; the table in
+    // tensor memory or in registers made the kernel alone slower, 35.4 against
+    // 34.4 us).
+    using WTab = WideWeightTable<TW, false>;
+    __shared__ uint32_t s_tmem;
+    if (ROUTE && warp == 0) {
+        tmem_alloc(&s_tmem, WTab::kCols);
+        tmem_relinquish();
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < NTEAM * nslot; ++i) mbar_init(&bars[i], 1);
         for (int i = 0; i < NTEAM; ++i) abort_all[4 * i] = 0;
         fence_mbar_init();
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     griddep_wait();     // inputs may come from the previous kernel on the stream
     griddep_launch();
-    if (team == 0) {
+    if constexpr (ROUTE) {
+        if (warp < 4) WTab::fill(s_tmem, warp, lane, a.w, 0.0f, lines);
+    } else if (team == 0) {
 #pragma unroll
         for (int c = 0; c < 8; ++c)
             wtab[c * P + tid] = has_line ? *reinterpret_cast<const uint4*>(a.w + 64 * tid + 8 * c)
                                          : make_uint4(0u, 0u, 0u, 0u);
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     if constexpr (ROUTE) {
         constexpr int RW = kFusedRouterWarps;
         if (warp >= NTEAM * TW) {
@@ -274,6 +295,7 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     const int team_stride = gridDim.x * NTEAM;
     uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
     const uint32_t ring_saddr = smem_addr(ring);
+    const uint32_t wt_taddr = ROUTE ? WTab::line_addr(s_tmem, warp, warp_in_team) : 0u;
     const uint32_t wtab_saddr = smem_addr(wtab);
     uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
     int* abort_word = abort_all + 4 * team;
@@ -358,14 +380,26 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
         pbuf ^= 1;
         const float inv = inv_rms_h(tree_sum_array<TW>(pp), fH, rH, pow2, a.eps);
         const float2 inv2 = make_float2(inv, inv);
-        if (has_line) {
+        if (ROUTE ? warp_has_line : has_line) {    // with the router warps every lane of the warp reads the table
         uint32_t codes[8];
         uint32_t sfw = 0u;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
-            const uint4 w0 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk) * P + tid));
-            const uint4 w1 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk + 1) * P + tid));
-            const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t ws[8];
+            if constexpr (ROUTE) {
+                tmem_ld8_ro(wt_taddr + 8u * static_cast<uint32_t>(blk), ws);
+            } else {
+                const uint4 w0 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk) * P + tid));
+                const uint4 w1 = lds128(wtab_saddr + 16u * static_cast<uint32_t>((2 * blk + 1) * P + tid));
+                ws[0] = w0.x;
+                ws[1] = w0.y;
+                ws[2] = w0.z;
+                ws[3] = w0.w;
+                ws[4] = w1.x;
+                ws[5] = w1.y;
+                ws[6] = w1.z;
+                ws[7] = w1.w;
+            }
             uint32_t yw[8];
             uint32_t m = 0u;
 #pragma unroll
@@ -393,15 +427,27 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
             codes[2 * blk + 1] = cvt_e2m1x8(q + 8);
             sfw |= sfc << (8 * blk);
         }
-        uint8_t* prow = a.packed + static_cast<size_t>(t) * (H / 2) + 32 * tid;
-        *reinterpret_cast<uint4*>(prow) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        *reinterpret_cast<uint4*>(prow + 16) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        *reinterpret_cast<uint32_t*>(a.sf + static_cast<size_t>(t) * nblocks + 4 * tid) = sfw;
+        if (has_line) {
+            uint8_t* prow = a.packed + static_cast<size_t>(t) * (H / 2) + 32 * tid;
+            *reinterpret_cast<uint4*>(prow) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            *reinterpret_cast<uint4*>(prow + 16) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            *reinterpret_cast<uint32_t*>(a.sf + static_cast<size_t>(t) * nblocks + 4 * tid) = sfw;
+        }
         }
     }
     if (tid == 0)
         for (int f = cur->consumed; f < cur->issued; ++f)
             mbar_wait_bounded(&tb[f % nslot], (f / nslot) & 1, 2u);
+    if constexpr (ROUTE) {
+        // the row warps (the router warps have left) release the weight table
+        // once every row warp's last read of it is done
+        tc_fence_before();
+        named_bar_sync(kTmemReleaseBar, NTEAM * P);
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(s_tmem, WTab::kCols);
+        }
+    }
 }
 
 namespace {

@@ -34,6 +34,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tmem.cuh"
 
 namespace mb {
 
@@ -93,6 +94,67 @@ struct WideLayout {
     __host__ __device__ size_t cursor_offset() const { return abort_offset() + static_cast<size_t>(nteam) * 16; }
     __host__ __device__ size_t total_bytes() const {
         return cursor_offset() + static_cast<size_t>(nteam) * sizeof(RingCursor) + kSlotAlign;
+    }
+};
+
+// The norm weights of a wide-row kernel in tensor memory.  Thread t of a team
+// owns line t (64 elements) of every row, and warp w of the CTA reaches lane
+// quadrant w % 4 only; since TW divides 4 or 4 divides TW, lane l of quadrant
+// g holds the weights of line 32 (g % TW) + l, and for TW = 8 a second column
+// block holds the lines of warps 4..7 of a team.  A line takes 32 columns of
+// packed BF16 pairs, or with GAINS 64 columns of the FP32 gains gc + w (formed
+// once, the same single rounding as forming them per row).  Lines past the
+// row's end hold zeros.
+template <int TW, bool GAINS>
+struct WideWeightTable {
+    static constexpr uint32_t kLineCols = GAINS ? 64u : 32u;
+    static constexpr int kColBlocks = TW > 4 ? 2 : 1;
+    static constexpr uint32_t kCols = kLineCols * kColBlocks;   // the allocation: 32..128 columns
+
+    // Warps 0..3 of the CTA fill it (each its own quadrant).
+    static __device__ __forceinline__ void fill(uint32_t base, int warp, int lane, const uint16_t* w, float gc,
+                                                int lines) {
+#pragma unroll
+        for (int cb = 0; cb < kColBlocks; ++cb) {
+            const int line = ((warp % TW) + 4 * cb) * 32 + lane;
+            const bool in = line < lines;
+            const uint32_t dst = base + ((32u * static_cast<uint32_t>(warp)) << 16) + kLineCols * cb;
+#pragma unroll
+            for (int h = 0; h < static_cast<int>(kLineCols / 32); ++h) {
+                uint32_t r[32];
+                if constexpr (!GAINS) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = in ? *reinterpret_cast<const uint4*>(w + 64 * line + 8 * c)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                        r[4 * c] = v.x;
+                        r[4 * c + 1] = v.y;
+                        r[4 * c + 2] = v.z;
+                        r[4 * c + 3] = v.w;
+                    }
+                } else {   // elements 32 h .. 32 h + 31 of the line
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = in ? *reinterpret_cast<const uint4*>(w + 64 * line + 32 * h + 8 * c)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float2 f = unpack_bf16x2(ws[q]);
+                            r[8 * c + 2 * q] = __float_as_uint(in ? __fadd_rn(gc, f.x) : 0.0f);
+                            r[8 * c + 2 * q + 1] = __float_as_uint(in ? __fadd_rn(gc, f.y) : 0.0f);
+                        }
+                    }
+                }
+                tmem_st32(dst + 32u * static_cast<uint32_t>(h), r);
+            }
+        }
+    }
+
+    // Address of this thread's line: its warp's quadrant, its column block.
+    static __device__ __forceinline__ uint32_t line_addr(uint32_t base, int warp, int warp_in_team) {
+        return base + ((32u * static_cast<uint32_t>(warp & 3)) << 16) +
+               kLineCols * static_cast<uint32_t>(warp_in_team >> 2);
     }
 };
 
