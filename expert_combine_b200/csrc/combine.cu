@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
     const int H = a.H;
     const int nslot = a.nslot;
     const int slot_bytes = slot_bytes_for(H);
-    const WideLayout lay{NTEAM, nslot, slot_bytes, P};
+    const WideLayout lay{NTEAM, nslot, slot_bytes, P, false};   // weights in tensor memory
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.bars_offset());
     float* part_all = reinterpret_cast<float*>(smem + lay.part_offset());
     int* abort_all = reinterpret_cast<int*>(smem + lay.abort_offset());
@@ -709,9 +709,13 @@ cudaError_t launch_wide(const CUtensorMap& tmap, const CombineArgs& args, cudaSt
     constexpr int P = TW * 32;
     constexpr int NTEAM = kConsumerThreads / P;
     const int slot_bytes = slot_bytes_for(args.H);
-    WideLayout lay{NTEAM, 1, slot_bytes, P};
+    WideLayout lay{NTEAM, 1, slot_bytes, P, false};
     const size_t fixed = lay.total_bytes() - static_cast<size_t>(NTEAM) * slot_bytes;
-    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - 64 * NTEAM;
+    cudaFuncAttributes fa{};   // the kernel's static shared memory counts against the same limit
+    cudaError_t fe = cudaFuncGetAttributes(&fa, combine_wide_kernel<TW, GC0>);
+    if (fe != cudaSuccess) return fe;
+    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - static_cast<int>(fa.sharedSizeBytes) -
+                      64 * NTEAM;
     int nslot = avail / (NTEAM * slot_bytes);
     if (nslot > 16) nslot = 16;
     if (nslot < 2) return cudaErrorInvalidConfiguration;

@@ -520,7 +520,11 @@ cudaError_t launch_nq_wide(const CUtensorMap& tmap, const NormQuantArgs& args, c
     const int slot_bytes = slot_bytes_for(args.H);
     WideLayout lay{NTEAM, 1, slot_bytes, P};
     const size_t fixed = lay.total_bytes() - static_cast<size_t>(NTEAM) * slot_bytes;
-    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - 64 * NTEAM;
+    cudaFuncAttributes fa{};   // the kernel's static shared memory counts against the same limit
+    cudaError_t fe = cudaFuncGetAttributes(&fa, norm_quant_wide_kernel<TW, GC0, ROUTE>);
+    if (fe != cudaSuccess) return fe;
+    const int avail = device_info().max_smem_optin - static_cast<int>(fixed) - static_cast<int>(fa.sharedSizeBytes) -
+                      64 * NTEAM;
     int nslot = avail / (NTEAM * slot_bytes);
     if (nslot > 16) nslot = 16;
     if (nslot < 2) return cudaErrorInvalidConfiguration;

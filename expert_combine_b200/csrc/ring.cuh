@@ -80,13 +80,17 @@ __host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a *
 __host__ __device__ inline int slot_bytes_for(int H) { return round_up(2 * H, kSlotAlign); }
 
 // Shared-memory carve-up of a wide-row CTA (one 128-byte line per thread):
-// row slots, the packed-weight table [8 chunks][P threads] x 16 B, slot
-// barriers, per-team partial buffers [2][TW], abort words and cursors.
+// row slots, the packed-weight table [8 chunks][P threads] x 16 B (only for a
+// kernel that reads its weights from shared memory: wtab), slot barriers,
+// per-team partial buffers [2][TW], abort words and cursors.
 struct WideLayout {
     int nteam, nslot, slot_bytes, P;
+    bool wtab = true;
     __host__ __device__ size_t slots_bytes() const { return static_cast<size_t>(nteam) * nslot * slot_bytes; }
     __host__ __device__ size_t wtab_offset() const { return slots_bytes(); }              // [8][P] x 16 B
-    __host__ __device__ size_t bars_offset() const { return wtab_offset() + static_cast<size_t>(P) * 128; }
+    __host__ __device__ size_t bars_offset() const {
+        return wtab_offset() + (wtab ? static_cast<size_t>(P) * 128 : 0);
+    }
     __host__ __device__ size_t part_offset() const {                                      // [nteam][2][TW] f32
         return (bars_offset() + static_cast<size_t>(nteam) * nslot * sizeof(uint64_t) + 15) & ~size_t(15);
     }
