@@ -270,6 +270,38 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
     tc_fence_after();
     griddep_wait();     // inputs may come from the previous kernel on the stream
     griddep_launch();
+
+    const int M = a.M;
+    const int team_stride = gridDim.x * NTEAM;
+    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
+    const uint32_t ring_saddr = smem_addr(ring);
+    const uint32_t wtab_saddr = smem_addr(wtab);
+    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
+    int* abort_word = abort_all + 4 * team;
+    float* part = part_all + team * 2 * TW;
+
+    // ---- the leader's copy cursor: one row (tp segments) per token
+    const int hs = H / a.tp;
+    const int seg_lines = hs / 64;
+    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
+    auto issue = [&]() {
+        const int nt = cur->ct;
+        if (nt >= M) return;
+        const int ws = cur->wslot;
+        mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
+        uint8_t* dst = ring + static_cast<size_t>(ws) * slot_bytes;
+        for (int s = 0; s < a.tp; ++s)
+            tma_load_2d(smem_addr(dst + static_cast<size_t>(s) * 2 * hs), &tmap, 0, (s * M + nt) * seg_lines,
+                        &tb[ws]);
+        cur->ct = nt + team_stride;
+        cur->issued += 1;
+        cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
+    };
+    // the row warps' leaders start their copies before the tables below are filled
+    if (warp < NTEAM * TW && tid == 0) {
+        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < nslot; ++i) issue();
+    }
     if constexpr (ROUTE) {
         if (warp < 4) WTab::fill(s_tmem, warp, lane, a.w, 0.0f, lines);
     } else if (team == 0) {
@@ -303,37 +335,7 @@ __global__ void __launch_bounds__(kConsumerThreads + (ROUTE ? 32 * kFusedRouterW
         }
     }
 
-    const int M = a.M;
-    const int team_stride = gridDim.x * NTEAM;
-    uint8_t* ring = smem + static_cast<size_t>(team) * nslot * slot_bytes;
-    const uint32_t ring_saddr = smem_addr(ring);
     const uint32_t wt_taddr = ROUTE ? WTab::line_addr(s_tmem, warp, warp_in_team) : 0u;
-    const uint32_t wtab_saddr = smem_addr(wtab);
-    uint64_t* tb = bars + static_cast<size_t>(team) * nslot;
-    int* abort_word = abort_all + 4 * team;
-    float* part = part_all + team * 2 * TW;
-
-    // ---- the leader's copy cursor: one row (tp segments) per token
-    const int hs = H / a.tp;
-    const int seg_lines = hs / 64;
-    RingCursor* cur = reinterpret_cast<RingCursor*>(smem + lay.cursor_offset()) + team;
-    auto issue = [&]() {
-        const int nt = cur->ct;
-        if (nt >= M) return;
-        const int ws = cur->wslot;
-        mbar_arrive_expect_tx(&tb[ws], 2u * static_cast<uint32_t>(H));
-        uint8_t* dst = ring + static_cast<size_t>(ws) * slot_bytes;
-        for (int s = 0; s < a.tp; ++s)
-            tma_load_2d(smem_addr(dst + static_cast<size_t>(s) * 2 * hs), &tmap, 0, (s * M + nt) * seg_lines,
-                        &tb[ws]);
-        cur->ct = nt + team_stride;
-        cur->issued += 1;
-        cur->wslot = (ws + 1 == nslot) ? 0 : ws + 1;
-    };
-    if (tid == 0) {
-        *cur = RingCursor{static_cast<int>(blockIdx.x) * NTEAM + team, 0, 0, 0, 0, 0, 0, 0};
-        for (int i = 0; i < nslot; ++i) issue();
-    }
 
     const float gs = __ldg(a.gs);
     const float rgs = __frcp_rn(gs);
