@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 // a team owns the 128-byte line t of every row (four 16-element blocks) and
 // keeps its 32 words in registers across the team barrier, so the slot is
 // refilled as soon as the barrier has passed.  The packed BF16 weights sit in
-// a shared-memory table read without bank conflicts.
+// a shared-memory table read without bank conflicts, or with ROUTE in tensor
+// memory (below).
 //
 // ROUTE: the CTA carries router warps after its row warps; they route the same
 // M tokens (one per warp iteration, statically interleaved over the grid's
