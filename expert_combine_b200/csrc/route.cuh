@@ -17,9 +17,10 @@
 // approximate score lies within twice the error bound below tau can belong to
 // the exact top k (every other one is exactly below k others).  Those
 // candidates -- typically k or a few more -- get the exact sigmoid, move to
-// one lane each and are ranked by broadcast, with no dependent chain of warp
-// reductions.  When more than 32 remain (massive exact ties) the token takes
-// the exact merge rounds over all its experts instead.
+// one lane each and are put in pick order by broadcast ranks or a bitonic
+// network across the lanes, with no dependent chain of warp reductions.  When more than 32 remain
+// (massive exact ties) the token takes the exact merge rounds over all its
+// experts instead.
 #pragma once
 
 #include "common.cuh"
@@ -295,13 +296,35 @@ __device__ __forceinline__ int nth_set_bit(uint32_t m, int n) {
     return pos;
 }
 
+// Largest expert id the shortlist's 64-bit order can carry (27 bits).
+constexpr uint32_t kShortlistIdMax = (1u << 27) - 1u;
+static_assert(kMaxExperts <= static_cast<int>(kShortlistIdMax) + 1, "expert ids fit the shortlist's order");
+
+// The warp's 64-bit values sorted descending over lanes 0..N-1 (N = 16 or 32;
+// lane l ends with the l-th largest): a bitonic network of compare-exchanges
+// between lanes l and l ^ stride, block l / size descending when even.
+template <int N>
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v, int lane) {
+#pragma unroll
+    for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+            const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+            v = keep_max ? (o > v ? o : v) : (o < v ? o : v);
+        }
+    }
+    return v;
+}
+
 // Rank a token's shortlisted experts exactly and write its picks.  Each lane
 // holds `cnt` of them; next_id() yields the lane's next expert id (cnt calls).
 // The ids move to one lane each, every lane computes its expert's exact
-// sigmoid and selection key at once, and the ranks come from broadcasts.
+// sigmoid and selection key at once, and broadcast ranks (up to 16) or a
+// bitonic network across the lanes (above) put them in pick order.
 // Returns false, writing nothing, when the warp holds more than 32 or fewer
 // than k shortlisted experts.
-template <class NextId>
+template <bool SORT32, class NextId>
 __device__ __forceinline__ bool shortlist_finish(int cnt, int lane, int k, NextId&& next_id,
                                                  const float* __restrict__ row, const float* __restrict__ bias,
                                                  int32_t* id_row, float* w_row) {
@@ -332,31 +355,45 @@ __device__ __forceinline__ bool shortlist_finish(int cnt, int lane, int k, NextI
         const uint32_t g = __shfl_sync(kAll, cid, src);
         if (rd == r) mid = g;
     }
-    // the order (key descending, id ascending) as one 64-bit number, larger first
+    // the order (key descending, id ascending) as one 64-bit number, larger
+    // first: key, then ~id -- or, for the network, 2^27 - 1 - id and the lane
+    // (ids are distinct, so the lane never decides; it tells where the
+    // candidate's sigmoid sits)
     uint64_t mine = 0u;                              // lanes without a candidate sort last
     float ms = 0.0f;
     if (lane < nc) {
         ms = sigmoid_fixed(__ldg(row + mid));
         const uint32_t key = score_key(__fadd_rn(ms, __ldg(bias + mid)));
-        mine = (static_cast<uint64_t>(key) << 32) | static_cast<uint64_t>(~mid);
+        mine = (static_cast<uint64_t>(key) << 32) |
+               (SORT32 ? (static_cast<uint64_t>(kShortlistIdMax - mid) << 5) | static_cast<uint64_t>(lane)
+                       : static_cast<uint64_t>(~mid));
     }
-    // rank: how many candidates come first; eight per step so that their
-    // broadcasts overlap
-    int rank = 0;
-    for (int i0 = 0; i0 < nc; i0 += 8) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const uint64_t other = __shfl_sync(kAll, mine, (i0 + q) & 31);
-            rank += (other > mine) ? 1 : 0;
-        }
-    }
-    // lane p learns which lane holds rank p: bit b of that lane's index, for
-    // every rank at once, in one warp OR per bit
+    // `from` on lane p: the lane holding the p-th largest.  With SORT32 and
+    // above 16 candidates a bitonic network over the 32 lanes sorts them (the
+    // lane travels in the low bits); otherwise each candidate's rank comes
+    // from broadcasts, eight per step so that they overlap, and lane p learns
+    // which lane holds rank p from one warp OR per bit of the lane index.  The
+    // network is cheaper at k = 22 (85.8 against 89.0 us at 65536 x 512); the
+    // broadcast ranks are cheaper up to 16 candidates (8.5 against 8.7 us at
+    // 8192 x 256, k = 8), and the large-E kernel, whose k is 8 in practice,
+    // runs faster without the network's code (115.5 against 118.2 us).
     int from = 0;
+    if (SORT32 && nc > 16) {
+        from = static_cast<int>(warp_sort_desc<32>(mine, lane) & 31u);
+    } else {
+        int rank = 0;
+        for (int i0 = 0; i0 < nc; i0 += 8) {
 #pragma unroll
-    for (int bit = 0; bit < 5; ++bit) {
-        const uint32_t m = __reduce_or_sync(kAll, (lane < nc && ((lane >> bit) & 1)) ? (1u << rank) : 0u);
-        from |= static_cast<int>((m >> lane) & 1u) << bit;
+            for (int q = 0; q < 8; ++q) {
+                const uint64_t other = __shfl_sync(kAll, mine, (i0 + q) & 31);
+                rank += (other > mine) ? 1 : 0;
+            }
+        }
+#pragma unroll
+        for (int bit = 0; bit < 5; ++bit) {
+            const uint32_t m = __reduce_or_sync(kAll, (lane < nc && ((lane >> bit) & 1)) ? (1u << rank) : 0u);
+            from |= static_cast<int>((m >> lane) & 1u) << bit;
+        }
     }
     const float sp = __shfl_sync(kAll, ms, from);    // lane p < k: the sigmoid of pick p
     const uint32_t idp = __shfl_sync(kAll, mid, from);
@@ -406,7 +443,7 @@ __device__ __forceinline__ bool route_token_shortlist(const float* __restrict__ 
         rem &= rem - 1u;
         return lane_pos_id(p, lane);
     };
-    return shortlist_finish(cnt, lane, k, next_id, row, bias, id_row, w_row);
+    return shortlist_finish<true>(cnt, lane, k, next_id, row, bias, id_row, w_row);
 }
 
 // Large E (more than 16 experts per lane): the fast scores go through the
@@ -524,7 +561,7 @@ __device__ __forceinline__ bool route_token_wide(const float* __restrict__ row, 
         for (int i = 1; i < kWideLaneCands; ++i) e = (q == i) ? cand[i] : e;
         return e;
     };
-    return shortlist_finish(cnt > kWideLaneCands ? 33 : cnt, lane, k, next_id, row, bias, id_row, w_row);
+    return shortlist_finish<false>(cnt > kWideLaneCands ? 33 : cnt, lane, k, next_id, row, bias, id_row, w_row);
 }
 
 // Exact merge rounds for the large-E path when its shortlist does not fit,
