@@ -371,8 +371,8 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 if (c / 2 < nvalid)
-                    *reinterpret_cast<uint4*>(orow + 8 * c) =
-                        make_uint4(brw[4 * c], brw[4 * c + 1], brw[4 * c + 2], brw[4 * c + 3]);
+                    __stcs(reinterpret_cast<uint4*>(orow + 8 * c),   // streaming: written once
+                           make_uint4(brw[4 * c], brw[4 * c + 1], brw[4 * c + 2], brw[4 * c + 3]));
         }
         if constexpr (JOIN) join_token32<TW>(brw, t, H, tid, nvalid, a.join, team_sum, pow2, rH);
     }
@@ -599,9 +599,9 @@ __global__ void __launch_bounds__(kConsumerThreads, 1)
             uint16_t* orow = a.out + static_cast<size_t>(t) * H + 64 * tid;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(orow + 8 * c) =
-                    make_uint4(pack_bf16x2_rn(acc[4 * c]), pack_bf16x2_rn(acc[4 * c + 1]),
-                               pack_bf16x2_rn(acc[4 * c + 2]), pack_bf16x2_rn(acc[4 * c + 3]));
+                __stcs(reinterpret_cast<uint4*>(orow + 8 * c),     // streaming: written once
+                       make_uint4(pack_bf16x2_rn(acc[4 * c]), pack_bf16x2_rn(acc[4 * c + 1]),
+                                  pack_bf16x2_rn(acc[4 * c + 2]), pack_bf16x2_rn(acc[4 * c + 3])));
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
