@@ -135,7 +135,7 @@ def test_combine_shapes(cuda_dev, H, k):
     check_combine(case)
 
 
-@pytest.mark.parametrize("H", [1024, 2688, 8192])
+@pytest.mark.parametrize("H", [1024, 2048, 2688, 8192, 16384])   # pair rows; wide rows of 1, 2 (partial), 4, 8 warps
 def test_combine_gain_centre_one(cuda_dev, H):
     case = synth.make_case("tiny", device=cuda_dev, T=29, H=H, join=False)
     g = torch.Generator(device=cuda_dev)
